@@ -1,0 +1,435 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 Strata MoE layer: MoE-layer tokens/s and % roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+                    [--workload NAME] [--layers L]
+
+A step is one forward of the whole layer (router -> top-k -> dispatch ->
+quantised SwiGLU experts -> combine) over one batch of T tokens.  Steps rotate
+over L independently seeded layers whose expert weights (L x 786 MB) exceed
+the 126 MB L2, so no step finds its weights in L2 ("inputs larger than L2").
+Each layer's forward is captured once in a CUDA graph and replayed.
+
+Multi-GPU (torchrun): each rank runs its own replica on its own tokens (the
+layer is token-parallel, so there is no data-path collective); `value` is the
+tokens of all ranks over the max-over-ranks device time (weak scaling).
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle (the
+plain C implementation the parity tests check against) on the host cores on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+WORKLOADS = {
+    # name: (shape, T, description)
+    "decode-t4": (gen.FLASH2, 4, "Flash-Next-shaped MoE layer, decode T=4 (MTP verify batch), "
+                                 "2-bit block-32"),
+    "decode-t1": (gen.FLASH2, 1, "Flash-Next-shaped MoE layer, decode T=1, 2-bit block-32"),
+    "decode3-t64": (gen.FLASH3, 64, "Flash-Next-shaped MoE layer, batched decode T=64, "
+                                    "3-bit block-32"),
+    "prefill-t8192": (gen.FLASH2, 8192, "Flash-Next-shaped MoE layer, prefill chunk T=8192, "
+                                        "2-bit block-32"),
+    "tiny-t8": (gen.TINY, 8, "tiny MoE layer H256 E16 k2 I64, T=8"),
+}
+DEFAULT_WORKLOAD = "decode-t4"
+STAGES = ["router", "topk", "dispatch", "gateup", "down", "combine"]
+GATEUP = 3
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period=0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as ex:  # no NVML: report nothing rather than guess
+            self.err = str(ex)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ helpers
+def expert_bytes(shape):
+    return shape.expert_bytes
+
+
+def mat_bytes(shape):
+    return shape.mat_code_bytes + 2 * shape.mat_scales
+
+
+def traffic_from_profile(workload):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu
+    summary, or None when the summary is missing or was taken on an older
+    version of the kernel source."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = os.path.join(ROOT, d.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if h != d.get("source_sha256"):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_throughput(layers, xs, shape, budget_s, threads):
+    """Tokens/s of the CPU oracle over (layer, token) jobs, bounded by budget_s."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = [(l, t) for t in range(xs[0].shape[0]) for l in range(len(layers))]
+    done = [0]
+    lock = threading.Lock()
+    t0 = time.perf_counter()
+
+    def work(j):
+        l, t = j
+        if time.perf_counter() - t0 > budget_s:
+            return
+        oracle.moe_forward(layers[l], xs[l], sel=np.array([t], dtype=np.int32))
+        with lock:
+            done[0] += 1
+
+    oracle.lib()
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, jobs))
+    dt = time.perf_counter() - t0
+    return done[0] / dt, done[0], dt
+
+
+def run_reference(args, wl):
+    """The reference arm: the CPU oracle on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    shape, T, desc = WORKLOADS[wl]
+    n_layers = min(args.layers, 4)
+    layers = [gen.layer_weights(shape, seed=0, layer=l) for l in range(n_layers)]
+    xs = [gen.hidden(T, shape.hidden, seed=100, layer=l) for l in range(n_layers)]
+    cores = os.cpu_count() or 1
+    import oracle
+    oracle.lib()
+    # warm-up: W steps, each one token through one layer (untimed; bounded)
+    budget = args.ref_budget
+    tw = time.perf_counter()
+    for i in range(min(args.warmup, 1)):
+        oracle.moe_forward(layers[0], xs[0], sel=np.array([0], dtype=np.int32))
+    del tw
+    # timed: up to K steps of one token through one layer, all host cores
+    from concurrent.futures import ThreadPoolExecutor
+    done = [0]
+    lock = threading.Lock()
+    t0 = time.perf_counter()
+
+    def step(i):
+        if time.perf_counter() - t0 > budget:
+            return
+        l = i % n_layers
+        t = (i // n_layers) % T
+        oracle.moe_forward(layers[l], xs[l], sel=np.array([t], dtype=np.int32))
+        with lock:
+            done[0] += 1
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(cores) as ex:
+        list(ex.map(step, range(args.steps)))
+    dt = time.perf_counter() - t0
+    value = done[0] / dt
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": done[0], "steps_requested": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1000 / max(done[0], 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl, "description": desc, "tokens_per_batch": T,
+                   "layers_rotated": n_layers},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{done[0]} steps of one token through one layer (routing + "
+                                   f"11 experts) across {n_layers} layers, {dt:.1f} s wall"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ own arm
+def run_own(args, wl):
+    import torch
+    import quantized_expert_ffn_04_b200 as qe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.cuda.current_device()
+    shape, T, desc = WORKLOADS[wl]
+    NL = args.layers
+    peaks, peak_kind = load_peaks()
+
+    # ---- layers (same weights on every rank, different tokens per rank)
+    host_layers = []
+    layers = []
+    for l in range(NL):
+        hw = gen.layer_weights(shape, seed=0, layer=l)
+        layers.append(qe.Layer(hw, max_tokens=T, device=dev))
+        if l < 2:
+            host_layers.append(hw)
+    xs_host = [gen.hidden(T, shape.hidden, seed=100 + rank, layer=l) for l in range(NL)]
+    xs = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).cuda() for x in xs_host]
+    ys = [torch.empty_like(x) for x in xs]
+    stream = torch.cuda.current_stream()
+
+    # ---- routing statistics for the algorithmic bytes (from the GPU's routing)
+    distinct = []
+    for l in range(NL):
+        idx, _, _, _ = layers[l].route(xs[l])
+        distinct.append(int(torch.unique(idx).numel()))
+    torch.cuda.synchronize()
+
+    # ---- probes around the dominant kernel (gate/up), one event pair per layer
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(NL)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(NL)]
+    for e in ev_b + ev_e:
+        e.record(stream)
+    torch.cuda.synchronize()
+    for l in range(NL):
+        qe.strata_moe_set_probe(layers[l].handle, GATEUP, ev_b[l].cuda_event, ev_e[l].cuda_event)
+
+    # ---- warm-up eagerly, then capture one graph per layer
+    for l in range(NL):
+        layers[l].forward(xs[l], out=ys[l], stream=stream)
+    torch.cuda.synchronize()
+    for l in range(NL):
+        layers[l].sync_status(stream)
+    graphs = []
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    for l in range(NL):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            layers[l].forward(xs[l], out=ys[l], stream=cap)
+        graphs.append(g)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        graphs[i % NL].replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+
+    # ---- timed region: exactly K steps
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clocks:
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            graphs[i % NL].replay()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    ms = t_start.elapsed_time(t_end)
+    for l in range(NL):
+        layers[l].sync_status(stream)
+    # dominant kernel: the last launch of each layer's graph inside the region
+    ran = sorted({i % NL for i in range(max(0, args.steps - NL), args.steps)})
+    gu_ms = [ev_b[l].elapsed_time(ev_e[l]) for l in ran]
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens = T * args.steps * world
+    value = tokens / (ms / 1000.0)
+
+    # ---- algorithmic bytes
+    mb = mat_bytes(shape)
+    gu_bytes = [(distinct[l] + 1) * 2 * mb + T * shape.hidden * 2 for l in ran]
+    achieved = sum(gu_bytes) / (sum(gu_ms) / 1000.0) / 1e9  # GB/s
+    peak = float(peaks["hbm_gbs"])
+    step_bytes = [shape.n_experts * shape.hidden * 4 + shape.n_experts * 4
+                  + (distinct[l] + 1) * shape.expert_bytes + 2 * T * shape.hidden * 2
+                  for l in range(NL)]
+
+    # ---- e2e through the host-buffer entry point (pinned host memory)
+    for l in range(NL):
+        qe.strata_moe_set_probe(layers[l].handle, GATEUP, None, None)
+    xh = [torch.from_numpy(x.view(np.int16).copy()).pin_memory() for x in xs_host]
+    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    e2e_steps = min(args.steps, args.e2e_steps)
+    for i in range(min(args.warmup, 8)):
+        qe.strata_moe_forward_host(layers[i % NL].handle, xh[i % NL].data_ptr(), T,
+                                   yh[i % NL].data_ptr(), stream.cuda_stream)
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        l = i % NL
+        qe.strata_moe_forward_host(layers[l].handle, xh[l].data_ptr(), T, yh[l].data_ptr(),
+                                   stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = T * e2e_steps * world / (e2e_ms / 1000.0)
+
+    # ---- CPU baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cores = os.cpu_count() or 1
+        v, n, dt = oracle_throughput(host_layers, xs_host[:len(host_layers)], shape,
+                                     args.cpu_budget, cores)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} (layer, token) forwards of the same workload (routing + "
+                         f"11 experts each) over {len(host_layers)} layers in {dt:.1f} s"}
+
+    launches = qe.strata_moe_launch_count(layers[0].handle, T) * args.steps
+    clk = clocks.summary()
+    line = {
+        "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl, "description": desc, "tokens_per_batch": T,
+                   "hidden": shape.hidden, "experts": shape.n_experts, "top_k": shape.top_k,
+                   "inter": shape.inter, "bits": shape.bits, "layers_rotated": NL,
+                   "l2": "inputs larger than L2: steps rotate over %d layers (%.1f GB of "
+                         "expert weights)" % (NL, NL * (shape.n_experts + 1)
+                                              * shape.expert_bytes / 1e9),
+                   "cuda_graphs": True, "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_gateup", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind,
+                     "traffic": traffic_from_profile(wl),
+                     "algorithmic_bytes_per_launch": statistics.mean(gu_bytes),
+                     "launch_ms": statistics.mean(gu_ms)},
+        "step_bytes": statistics.mean(step_bytes),
+        "step_hbm_frac": statistics.mean(step_bytes) / (ms_step / 1000.0) / 1e9 / peak,
+        "distinct_experts": statistics.mean(distinct),
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.hidden * 2,
+                "d2h_bytes_per_step": T * shape.hidden * 2, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+    }
+    for g in graphs:
+        del g
+    graphs.clear()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=1000)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, args.workload)
+    else:
+        run_own(args, args.workload)
+
+
+if __name__ == "__main__":
+    main()

@@ -141,13 +141,27 @@ def dequant_rows(codes_m, scales_m, bits: int, cols: int, row0: int, nrows: int)
 
 
 # ---------------------------------------------------------------- routing
-def router_logits(x_bits: np.ndarray, W: np.ndarray, b: np.ndarray | None) -> np.ndarray:
+def router_logits(x_bits: np.ndarray, W: np.ndarray, b: np.ndarray | None,
+                  threads: int = 1) -> np.ndarray:
+    """fp32 logits [T, E]; `threads` > 1 splits the tokens across threads."""
     x_bits, W = _c(x_bits, np.uint16), _c(W, np.float32)
     T, H = x_bits.shape
     E = W.shape[0]
     b = None if b is None else _c(b, np.float32)
     out = np.empty((T, E), dtype=np.float32)
-    lib().orc_router_logits(_p(x_bits), T, H, _p(W), _p(b), E, _p(out))
+    L = lib()
+
+    def run(lo, hi):
+        if hi > lo:
+            L.orc_router_logits(_p(x_bits[lo:hi]), hi - lo, H, _p(W), _p(b), E, _p(out[lo:hi]))
+
+    threads = max(1, min(threads, T))
+    bounds = np.linspace(0, T, threads + 1).astype(int)
+    if threads == 1:
+        run(0, T)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: run(bounds[i], bounds[i + 1]), range(threads)))
     return out
 
 

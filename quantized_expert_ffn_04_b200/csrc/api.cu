@@ -1,0 +1,563 @@
+// C ABI of the Strata MoE layer library: handle lifetime, weight upload and
+// repack, and the per-call orchestration of the kernels on the caller's
+// stream.  Every step of the layer runs in this library's kernels; there is no
+// host fallback.
+#include <cuda_runtime.h>
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/strata_moe.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace strata;
+
+namespace {
+
+thread_local std::string g_err;
+
+strata_status fail(strata_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+strata_status fail(strata_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+strata_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(STRATA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Switch to a device for the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+constexpr long long kDefaultBudget = 4000000000ll;  // ~2 s at the top SM clock
+
+}  // namespace
+
+struct strata_moe {
+    int device = 0;
+    strata_moe_config cfg{};
+    Geometry geo{};
+    uint8_t *wq = nullptr;        // (E + 1) experts; the shared expert last
+    float *router_wp = nullptr;   // [E][H/128][32][4]
+    float *router_b = nullptr;    // [E] or null
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    // workspace views
+    float *logits = nullptr;
+    int32_t *idx = nullptr, *slot = nullptr, *list = nullptr, *cnt = nullptr, *off = nullptr;
+    float *wts = nullptr;
+    DispatchScratch ds{};
+    int4 *units = nullptr;
+    int *n_units = nullptr;
+    void *a = nullptr;            // fp16 [slots][Ip]
+    void *Y = nullptr;            // fp32 (decode) / fp16 (prefill) [slots][H]
+    int *err = nullptr;
+    void *xio = nullptr, *yio = nullptr, *xn = nullptr;  // bf16 [max_tokens][H]
+    cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
+    // options
+    int path = 0;
+    long long budget = kDefaultBudget;
+    int decode_max_t = 64;
+};
+
+namespace {
+
+strata_status validate_config(const strata_moe_config *c) {
+    if (!c) return fail(STRATA_ERR_INVALID_ARG, "config is NULL");
+    if (c->hidden <= 0 || c->n_experts <= 0 || c->top_k <= 0 || c->inter <= 0 ||
+        c->max_tokens <= 0 || c->block <= 0)
+        return fail(STRATA_ERR_INVALID_ARG, "config fields must be positive");
+    if (c->block != 32) return fail(STRATA_ERR_UNSUPPORTED, "block must be 32 (got %d)", c->block);
+    if (c->quant_bits != 2 && c->quant_bits != 3)
+        return fail(STRATA_ERR_UNSUPPORTED, "quant_bits must be 2 or 3 (got %d)", c->quant_bits);
+    if (c->hidden % 128 || c->hidden > 6144)
+        return fail(STRATA_ERR_UNSUPPORTED, "hidden must be a multiple of 128 and <= 6144 (got %d)",
+                    c->hidden);
+    if (c->inter % 32 || c->inter > 4096)
+        return fail(STRATA_ERR_UNSUPPORTED, "inter must be a multiple of 32 and <= 4096 (got %d)",
+                    c->inter);
+    if (c->n_experts > 1024)
+        return fail(STRATA_ERR_UNSUPPORTED, "n_experts must be <= 1024 (got %d)", c->n_experts);
+    if (c->top_k > c->n_experts || c->top_k > 32)
+        return fail(STRATA_ERR_UNSUPPORTED, "top_k must be <= min(n_experts, 32) (got %d)",
+                    c->top_k);
+    if (c->max_tokens > 65536)
+        return fail(STRATA_ERR_UNSUPPORTED, "max_tokens must be <= 65536 (got %d)",
+                    c->max_tokens);
+    return STRATA_OK;
+}
+
+Geometry make_geometry(const strata_moe_config &c) {
+    Geometry g{};
+    g.H = c.hidden;
+    g.E = c.n_experts;
+    g.k = c.top_k;
+    g.I = c.inter;
+    g.Ip = (c.inter + 127) / 128 * 128;
+    g.bits = c.quant_bits;
+    g.nseg_h = g.H / kSegCols;
+    g.nseg_i = g.Ip / kSegCols;
+    g.ub = unit_bytes(g.bits);
+    g.mat_bytes = (size_t)(g.Ip / kSlabRows) * g.nseg_h * g.ub;
+    g.expert_bytes = 3 * g.mat_bytes;
+    return g;
+}
+
+// Carve the workspace; with base == nullptr only computes the size.
+size_t carve_workspace(strata_moe *h, char *base) {
+    const Geometry &g = h->geo;
+    const size_t T = (size_t)h->cfg.max_tokens, k = g.k, E = g.E, H = g.H;
+    const size_t slots = T * k + T;
+    const size_t y_bytes = slots * H * 4;  // fp32 staging of every (slot, column)
+    int units = max_units((int)T, (int)k, (int)E, 8);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return base ? base + o : nullptr;
+    };
+    h->logits = (float *)take(T * E * 4);
+    h->idx = (int32_t *)take(T * k * 4);
+    h->wts = (float *)take(T * k * 4);
+    h->slot = (int32_t *)take(T * k * 4);
+    h->list = (int32_t *)take(T * k * 4);
+    h->cnt = (int32_t *)take(E * 4);
+    h->off = (int32_t *)take((E + 1) * 4);
+    char *dsb = take(dispatch_scratch_bytes((int)T, (int)E));
+    if (base) dispatch_scratch_carve(dsb, (int)T, (int)E, &h->ds);
+    h->units = (int4 *)take((size_t)units * 16);
+    h->n_units = (int *)take(4);
+    h->err = (int *)take(4);
+    h->a = take(slots * g.Ip * 2);
+    h->Y = take(y_bytes);
+    h->xio = take(T * H * 2);
+    h->yio = take(T * H * 2);
+    h->xn = take(T * H * 2);
+    return off;
+}
+
+void free_handle(strata_moe *h) {
+    if (!h) return;
+    cudaFree(h->wq);
+    cudaFree(h->router_wp);
+    cudaFree(h->router_b);
+    cudaFree(h->ws);
+    delete h;
+}
+
+strata_status check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return STRATA_OK;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const char *pa = (const char *)a, *pb = (const char *)b;
+    return pa < pb + nb && pb < pa + na;
+}
+
+strata_status check_tokens(strata_moe_t h, int T) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(STRATA_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+    if (T > h->cfg.max_tokens)
+        return fail(STRATA_ERR_INVALID_ARG, "T = %d exceeds max_tokens = %d", T,
+                    h->cfg.max_tokens);
+    return STRATA_OK;
+}
+
+enum { kStRouter, kStTopk, kStDispatch, kStGateUp, kStDown, kStCombine };
+
+void probe(strata_moe_t h, int stage, bool begin, cudaStream_t s) {
+    cudaEvent_t e = begin ? h->probe_begin[stage] : h->probe_end[stage];
+    if (e) cudaEventRecord(e, s);
+}
+
+// Router + top-k + dispatch into the handle's workspace.
+strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStream_t s) {
+    const Geometry &g = h->geo;
+    probe(h, kStRouter, true, s);
+    launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s);
+    probe(h, kStRouter, false, s);
+    probe(h, kStTopk, true, s);
+    launch_topk(h->logits, T, g.E, g.k, h->idx, h->wts, s);
+    probe(h, kStTopk, false, s);
+    probe(h, kStDispatch, true, s);
+    launch_dispatch(h->idx, T, g.k, g.E, h->cnt, h->off, h->list, h->slot, h->ds, h->units,
+                    h->n_units, tile, s);
+    probe(h, kStDispatch, false, s);
+    return check_launch("routing kernels");
+}
+
+strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool residual,
+                          cudaStream_t s) {
+    const Geometry &g = h->geo;
+    strata_status st = run_route(h, x, T, 8, s);
+    if (st != STRATA_OK) return st;
+    ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
+    int umax = max_units(T, g.k, g.E, 8);
+    probe(h, kStGateUp, true, s);
+    launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->a, h->err,
+                       h->budget, s);
+    probe(h, kStGateUp, false, s);
+    probe(h, kStDown, true, s);
+    launch_gemv_down(g, w, h->units, h->n_units, umax, h->a, (float *)h->Y, h->err, h->budget,
+                     s);
+    probe(h, kStDown, false, s);
+    probe(h, kStCombine, true, s);
+    launch_combine(h->Y, false, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s);
+    probe(h, kStCombine, false, s);
+    return check_launch("expert kernels");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *strata_moe_last_error(void) { return g_err.c_str(); }
+
+const char *strata_moe_version(void) { return "strata-moe-b200 0.1 (sm_100a)"; }
+
+strata_status strata_moe_set_probe(strata_moe_t h, int stage, void *ev_begin, void *ev_end) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    if (stage < 0 || stage > 5) return fail(STRATA_ERR_INVALID_ARG, "stage must be 0..5");
+    h->probe_begin[stage] = (cudaEvent_t)ev_begin;
+    h->probe_end[stage] = (cudaEvent_t)ev_end;
+    return STRATA_OK;
+}
+
+int strata_moe_launch_count(strata_moe_t h, int T) {
+    if (!h || T < 0 || T > h->cfg.max_tokens) return 0;
+    if (T == 0) return 0;
+    return 3 /* router, top-k, combine */ + 3 /* dispatch */ + 2 /* gate/up, down */;
+}
+
+strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_weights *wts,
+                                int device, strata_moe_t *out) {
+    if (!out) return fail(STRATA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    strata_status st = validate_config(cfg);
+    if (st != STRATA_OK) return st;
+    if (!wts || !wts->codes || !wts->scales || !wts->router_w || !wts->shared_codes ||
+        !wts->shared_scales || (cfg->has_router_bias && !wts->router_b))
+        return fail(STRATA_ERR_INVALID_ARG, "a required weight pointer is NULL");
+    int ndev = 0;
+    cudaError_t ce = cudaGetDeviceCount(&ndev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDeviceCount");
+    if (device < 0 || device >= ndev)
+        return fail(STRATA_ERR_INVALID_ARG, "device %d out of range (%d devices)", device, ndev);
+    DeviceGuard guard(device);
+    if (!guard.ok) return fail(STRATA_ERR_CUDA, "cudaSetDevice(%d) failed", device);
+
+    if ((ce = init_kernel_attributes()) != cudaSuccess)
+        return cuda_fail(ce, "kernel attribute setup");
+    strata_moe *h = new strata_moe();
+    h->device = device;
+    h->cfg = *cfg;
+    h->geo = make_geometry(*cfg);
+    const Geometry &g = h->geo;
+    const size_t H = g.H, E = g.E;
+
+    // ---- allocations
+    size_t ws_bytes = carve_workspace(h, nullptr);
+    if (cudaMalloc(&h->wq, (E + 1) * g.expert_bytes) != cudaSuccess ||
+        cudaMalloc(&h->router_wp, E * H * 4) != cudaSuccess ||
+        (cfg->has_router_bias && cudaMalloc(&h->router_b, E * 4) != cudaSuccess) ||
+        cudaMalloc(&h->ws, ws_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        size_t wbytes = (E + 1) * g.expert_bytes;
+        free_handle(h);
+        return fail(STRATA_ERR_OOM, "device allocation failed (weights %zu B, workspace %zu B)",
+                    wbytes, ws_bytes);
+    }
+    h->ws_bytes = ws_bytes;
+    carve_workspace(h, (char *)h->ws);
+    if ((ce = cudaMemset(h->ws, 0, ws_bytes)) != cudaSuccess) {
+        free_handle(h);
+        return cuda_fail(ce, "cudaMemset(workspace)");
+    }
+
+    // ---- router: lane-interleaved copy of W (Wp[e][s4][l][j] = W[e][128 s4 + 32 j + l])
+    {
+        std::vector<float> wp(E * H);
+        for (size_t e = 0; e < E; e++)
+            for (size_t i = 0; i < H; i++) {
+                size_t s4 = i / 128, j = (i / 32) % 4, l = i % 32;
+                wp[((e * (H / 128) + s4) * 32 + l) * 4 + j] = wts->router_w[e * H + i];
+            }
+        ce = cudaMemcpy(h->router_wp, wp.data(), E * H * 4, cudaMemcpyHostToDevice);
+        if (ce == cudaSuccess && cfg->has_router_bias)
+            ce = cudaMemcpy(h->router_b, wts->router_b, E * 4, cudaMemcpyHostToDevice);
+        if (ce != cudaSuccess) {
+            free_handle(h);
+            return cuda_fail(ce, "router upload");
+        }
+    }
+
+    // ---- experts: upload the canonical format in batches, repack on the device
+    {
+        const size_t mat_codes = H * g.I * g.bits / 8, mat_scales = H * g.I / 32;
+        const size_t ex_codes = 3 * mat_codes, ex_scales = 3 * mat_scales;
+        const size_t batch = 32;
+        uint8_t *tc = nullptr;
+        uint16_t *ts = nullptr;
+        if (cudaMalloc(&tc, batch * ex_codes) != cudaSuccess ||
+            cudaMalloc(&ts, batch * ex_scales * 2) != cudaSuccess) {
+            cudaGetLastError();
+            cudaFree(tc);
+            free_handle(h);
+            return fail(STRATA_ERR_OOM, "staging allocation failed");
+        }
+        for (size_t e0 = 0; e0 <= E && ce == cudaSuccess; e0 += batch) {
+            size_t nb = (E + 1 - e0) < batch ? (E + 1 - e0) : batch;  // expert E = shared
+            for (size_t i = 0; i < nb && ce == cudaSuccess; i++) {
+                size_t e = e0 + i;
+                const uint8_t *src_c = e < E ? wts->codes + e * ex_codes : wts->shared_codes;
+                const uint16_t *src_s = e < E ? wts->scales + e * ex_scales : wts->shared_scales;
+                ce = cudaMemcpy(tc + i * ex_codes, src_c, ex_codes, cudaMemcpyHostToDevice);
+                if (ce == cudaSuccess)
+                    ce = cudaMemcpy(ts + i * ex_scales, src_s, ex_scales * 2,
+                                    cudaMemcpyHostToDevice);
+            }
+            for (size_t i = 0; i < nb && ce == cudaSuccess; i++) {
+                uint8_t *dst = h->wq + (e0 + i) * g.expert_bytes;
+                for (int m = 0; m < 3; m++) {
+                    const uint8_t *c = tc + i * ex_codes + m * mat_codes;
+                    const uint16_t *s = ts + i * ex_scales + m * mat_scales;
+                    if (m < 2)
+                        launch_repack_matrix(c, s, g.bits, g.I, g.H, g.Ip, g.H,
+                                             dst + m * g.mat_bytes, 0);
+                    else
+                        launch_repack_matrix(c, s, g.bits, g.H, g.I, g.H, g.Ip,
+                                             dst + m * g.mat_bytes, 0);
+                }
+                ce = cudaGetLastError();
+            }
+            if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+        }
+        cudaFree(tc);
+        cudaFree(ts);
+        if (ce != cudaSuccess) {
+            free_handle(h);
+            return cuda_fail(ce, "expert upload / repack");
+        }
+    }
+    *out = h;
+    return STRATA_OK;
+}
+
+void strata_moe_destroy(strata_moe_t h) {
+    if (!h) return;
+    DeviceGuard guard(h->device);
+    cudaDeviceSynchronize();
+    free_handle(h);
+}
+
+strata_status strata_moe_set_option(strata_moe_t h, int option, int64_t value) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    switch (option) {
+    case STRATA_OPT_PATH:
+        if (value < 0 || value > 2) return fail(STRATA_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+        h->path = (int)value;
+        return STRATA_OK;
+    case STRATA_OPT_WAIT_BUDGET:
+        if (value < 0) return fail(STRATA_ERR_INVALID_ARG, "wait budget must be >= 0");
+        h->budget = value;
+        return STRATA_OK;
+    case STRATA_OPT_DECODE_MAX_T:
+        if (value < 0) return fail(STRATA_ERR_INVALID_ARG, "decode max T must be >= 0");
+        h->decode_max_t = (int)value;
+        return STRATA_OK;
+    default:
+        return fail(STRATA_ERR_INVALID_ARG, "unknown option %d", option);
+    }
+}
+
+strata_status strata_moe_route(strata_moe_t h, const void *x_dev, int T, int32_t *idx_dev,
+                               float *w_dev, int32_t *offsets_dev, int32_t *list_dev,
+                               void *stream) {
+    strata_status st = check_tokens(h, T);
+    if (st != STRATA_OK) return st;
+    if (T == 0) return STRATA_OK;
+    if (!x_dev || !idx_dev || !w_dev) return fail(STRATA_ERR_INVALID_ARG, "NULL device pointer");
+    if (((uintptr_t)x_dev) & 15) return fail(STRATA_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    DeviceGuard guard(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Geometry &g = h->geo;
+    st = run_route(h, x_dev, T, 8, s);
+    if (st != STRATA_OK) return st;
+    cudaError_t ce;
+    size_t tk = (size_t)T * g.k;
+    if ((ce = cudaMemcpyAsync(idx_dev, h->idx, tk * 4, cudaMemcpyDeviceToDevice, s)) ||
+        (ce = cudaMemcpyAsync(w_dev, h->wts, tk * 4, cudaMemcpyDeviceToDevice, s)) ||
+        (offsets_dev &&
+         (ce = cudaMemcpyAsync(offsets_dev, h->off, (g.E + 1) * 4, cudaMemcpyDeviceToDevice, s))) ||
+        (list_dev && (ce = cudaMemcpyAsync(list_dev, h->list, tk * 4, cudaMemcpyDeviceToDevice, s))))
+        return cuda_fail(ce, "route output copy");
+    return STRATA_OK;
+}
+
+strata_status strata_moe_forward(strata_moe_t h, const void *x_dev, int T, void *y_dev,
+                                 void *stream) {
+    strata_status st = check_tokens(h, T);
+    if (st != STRATA_OK) return st;
+    if (T == 0) return STRATA_OK;
+    if (!x_dev || !y_dev) return fail(STRATA_ERR_INVALID_ARG, "NULL device pointer");
+    size_t bytes = (size_t)T * h->geo.H * 2;
+    if (overlaps(x_dev, bytes, y_dev, bytes))
+        return fail(STRATA_ERR_INVALID_ARG, "x and y overlap");
+    if ((((uintptr_t)x_dev) | ((uintptr_t)y_dev)) & 15)
+        return fail(STRATA_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+    DeviceGuard guard(h->device);
+    return run_forward(h, x_dev, T, y_dev, false, (cudaStream_t)stream);
+}
+
+strata_status strata_moe_sync_status(strata_moe_t h, void *stream) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    DeviceGuard guard(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t ce = cudaStreamSynchronize(s);
+    if (ce != cudaSuccess) return cuda_fail(ce, "stream synchronize");
+    int e = 0;
+    ce = cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost);
+    if (ce != cudaSuccess) return cuda_fail(ce, "error word read");
+    if (e) {
+        int z = 0;
+        cudaMemcpy(h->err, &z, 4, cudaMemcpyHostToDevice);
+        return fail(STRATA_ERR_TIMEOUT, "a device-side wait gave up (code %d)", e);
+    }
+    return STRATA_OK;
+}
+
+strata_status strata_moe_forward_host(strata_moe_t h, const void *x_host, int T, void *y_host,
+                                      void *stream) {
+    strata_status st = check_tokens(h, T);
+    if (st != STRATA_OK) return st;
+    if (T == 0) return STRATA_OK;
+    if (!x_host || !y_host) return fail(STRATA_ERR_INVALID_ARG, "NULL host pointer");
+    DeviceGuard guard(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    size_t bytes = (size_t)T * h->geo.H * 2;
+    cudaError_t ce = cudaMemcpyAsync(h->xio, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (ce != cudaSuccess) return cuda_fail(ce, "host to device copy");
+    st = run_forward(h, h->xio, T, h->yio, false, s);
+    if (st != STRATA_OK) return st;
+    ce = cudaMemcpyAsync(y_host, h->yio, bytes, cudaMemcpyDeviceToHost, s);
+    if (ce != cudaSuccess) return cuda_fail(ce, "device to host copy");
+    return strata_moe_sync_status(h, stream);
+}
+
+strata_status strata_moe_rmsnorm(const void *h_dev, void *xn_dev, int T, int H, void *stream) {
+    if (T < 0 || H <= 0 || H % 32) return fail(STRATA_ERR_INVALID_ARG, "bad T or H");
+    if (T == 0) return STRATA_OK;
+    if (!h_dev || !xn_dev) return fail(STRATA_ERR_INVALID_ARG, "NULL device pointer");
+    if (overlaps(h_dev, (size_t)T * H * 2, xn_dev, (size_t)T * H * 2))
+        return fail(STRATA_ERR_INVALID_ARG, "h and xn overlap");
+    launch_rmsnorm(h_dev, xn_dev, T, H, (cudaStream_t)stream);
+    return check_launch("rmsnorm");
+}
+
+strata_status strata_moe_stack_forward(const strata_moe_t *layers, int n_layers, void *h_dev,
+                                       int T, void *h_trace_dev, void *stream) {
+    if (!layers || n_layers <= 0) return fail(STRATA_ERR_INVALID_ARG, "no layers");
+    strata_moe_t l0 = layers[0];
+    strata_status st = check_tokens(l0, T);
+    if (st != STRATA_OK) return st;
+    if (T == 0) return STRATA_OK;
+    if (!h_dev) return fail(STRATA_ERR_INVALID_ARG, "h is NULL");
+    for (int l = 0; l < n_layers; l++) {
+        strata_moe_t L = layers[l];
+        if (!L || L->device != l0->device || L->cfg.hidden != l0->cfg.hidden ||
+            L->cfg.n_experts != l0->cfg.n_experts || L->cfg.top_k != l0->cfg.top_k ||
+            L->cfg.inter != l0->cfg.inter || L->cfg.quant_bits != l0->cfg.quant_bits)
+            return fail(STRATA_ERR_INVALID_ARG, "layer %d does not match layer 0", l);
+    }
+    DeviceGuard guard(l0->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t bytes = (size_t)T * l0->geo.H * 2;
+    for (int l = 0; l < n_layers; l++) {
+        strata_moe_t L = layers[l];
+        if (h_trace_dev) {
+            cudaError_t ce = cudaMemcpyAsync((char *)h_trace_dev + l * bytes, h_dev, bytes,
+                                             cudaMemcpyDeviceToDevice, s);
+            if (ce != cudaSuccess) return cuda_fail(ce, "trace copy");
+        }
+        launch_rmsnorm(h_dev, l0->xn, T, l0->geo.H, s);
+        // run layer L's weights in layer 0's workspace
+        strata_moe view = *l0;
+        view.wq = L->wq;
+        view.router_wp = L->router_wp;
+        view.router_b = L->router_b;
+        view.cfg.has_router_bias = L->cfg.has_router_bias;
+        st = run_forward(&view, l0->xn, T, h_dev, true, s);
+        if (st != STRATA_OK) return st;
+    }
+    return STRATA_OK;
+}
+
+strata_status strata_moe_debug_dequant(strata_moe_t h, int expert, int mat, int row0, int nrows,
+                                       int kind, float *out_host) {
+    if (!h || !out_host) return fail(STRATA_ERR_INVALID_ARG, "NULL argument");
+    const Geometry &g = h->geo;
+    if (expert < -1 || expert >= g.E || mat < 0 || mat > 2 || (kind != 0 && kind != 1))
+        return fail(STRATA_ERR_INVALID_ARG, "bad expert, mat or kind");
+    int rows = mat < 2 ? g.I : g.H, cols = mat < 2 ? g.H : g.I, Kp = mat < 2 ? g.H : g.Ip;
+    if (row0 < 0 || nrows <= 0 || row0 + nrows > rows)
+        return fail(STRATA_ERR_INVALID_ARG, "row range out of bounds");
+    DeviceGuard guard(h->device);
+    size_t e = expert < 0 ? (size_t)g.E : (size_t)expert;
+    const uint8_t *m = h->wq + e * g.expert_bytes + mat * g.mat_bytes;
+    float *d = nullptr;
+    size_t n = (size_t)nrows * cols;
+    cudaError_t ce = cudaMalloc(&d, n * 4);
+    if (ce != cudaSuccess) return fail(STRATA_ERR_OOM, "debug buffer");
+    launch_debug_dequant(m, g.bits, Kp, row0, nrows, cols, kind, d, 0);
+    ce = cudaGetLastError();
+    if (ce == cudaSuccess) ce = cudaMemcpy(out_host, d, n * 4, cudaMemcpyDeviceToHost);
+    cudaFree(d);
+    if (ce != cudaSuccess) return cuda_fail(ce, "debug dequant");
+    return STRATA_OK;
+}
+
+strata_status strata_moe_selftest_wait(int device, int64_t budget_cycles) {
+    int ndev = 0;
+    cudaError_t ce = cudaGetDeviceCount(&ndev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDeviceCount");
+    if (device < 0 || device >= ndev) return fail(STRATA_ERR_INVALID_ARG, "bad device");
+    DeviceGuard guard(device);
+    int *err = nullptr;
+    if (cudaMalloc(&err, 4) != cudaSuccess) return fail(STRATA_ERR_OOM, "selftest buffer");
+    cudaMemset(err, 0, 4);
+    launch_selftest_wait(err, budget_cycles, 0);
+    int e = 0;
+    ce = cudaGetLastError();
+    if (ce == cudaSuccess) ce = cudaMemcpy(&e, err, 4, cudaMemcpyDeviceToHost);
+    cudaFree(err);
+    if (ce != cudaSuccess) return cuda_fail(ce, "selftest");
+    if (e) return fail(STRATA_ERR_TIMEOUT, "the bounded wait gave up as designed");
+    return STRATA_OK;
+}
+
+}  // extern "C"

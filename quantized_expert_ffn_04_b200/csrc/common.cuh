@@ -1,0 +1,199 @@
+// Device helpers shared by the library's kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define STRATA_DEV __device__ __forceinline__
+
+namespace strata {
+
+// ---------------------------------------------------------------- layout
+// GPU weight layout of one quantised matrix [R rows][K cols]:
+//   slabs of 16 rows x segments of 128 columns; unit (slab, seg) at
+//   ((slab * (K/128)) + seg) * unit_bytes.  Inside a unit:
+//     [0, 512)        low two bits of every code, mma-fragment order:
+//                     lane L = 4g + c owns 16 bytes = 4 words, word w = block w
+//                     of the segment (32 columns).  Bit positions inside word w
+//                     for fragment register r' = 4s + r (s = k-step of the block,
+//                     r = mma A register 0..3): half 0 at bits 2r'..2r'+1,
+//                     half 1 at bits 16+2r'..16+2r'+1.
+//                     Register r holds (row, col) pairs of the m16n8k16 A
+//                     fragment: r=0 (g, 2c|2c+1), r=1 (g+8, 2c|2c+1),
+//                     r=2 (g, 2c+8|2c+9), r=3 (g+8, 2c+8|2c+9); col relative to
+//                     16*s inside the block.
+//     [512, 768)      3-bit only: high bit of every code, lane L owns 8 bytes =
+//                     2 words; word h holds blocks 2h (bits r', 16+r') and
+//                     2h+1 (bits 8+r', 24+r').
+//     [.., +128)      scales: lane L = 4g + c owns {d[g][c], d[g+8][c]} (fp16).
+constexpr int kSlabRows = 16;
+constexpr int kSegCols = 128;
+constexpr int kLoBytes = 512;
+constexpr int kHiBytes = 256;
+constexpr int kScaleBytes = 128;
+
+__host__ __device__ constexpr int unit_bytes(int bits) {
+    return kLoBytes + (bits == 3 ? kHiBytes : 0) + kScaleBytes;
+}
+
+// ---------------------------------------------------------------- errors
+// Device error word codes (handle workspace).
+constexpr int kErrTimeout = 1;
+
+// ---------------------------------------------------------------- smem / PTX
+STRATA_DEV uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+STRATA_DEV void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+STRATA_DEV void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+STRATA_DEV void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+STRATA_DEV void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+STRATA_DEV void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+STRATA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar`, giving up after `budget` SM cycles.  On
+// give-up the handle's error word gets kErrTimeout and false is returned.
+STRATA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget, int *err) {
+    if (budget <= 0) {
+        if (err) atomicCAS(err, 0, kErrTimeout);
+        return false;
+    }
+    long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > budget) {
+            if (err) atomicCAS(err, 0, kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// After a wait gave up: let the copies this barrier tracks land before the
+// CTA exits (bounded by a fixed, generous limit).
+constexpr long long kDrainCycles = 1ll << 31;
+STRATA_DEV void mbar_drain(uint64_t *bar, uint32_t parity) {
+    long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kDrainCycles) return;
+    }
+}
+
+// 1-D bulk copy global -> shared (no multicast), completes tx on `bar`.
+// dst, src 16-byte aligned, bytes a multiple of 16.
+STRATA_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+STRATA_DEV void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                            const void *smem_row) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(smem_row)));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
+STRATA_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                         const float (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+          "f"(c[2]), "f"(c[3]));
+}
+
+STRATA_DEV void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                        const float (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+          "f"(c[2]), "f"(c[3]));
+}
+
+// ---------------------------------------------------------------- dequant
+// Exact integer operand 2q - (2^bits - 1) in a 16-bit float lane pair, from the
+// GPU layout's code words.  The magic exponent leaves an ulp of 1, so OR-ing
+// 2q into the mantissa gives M + 2q exactly; subtracting M + 2^bits - 1 (exact)
+// leaves the odd integer 2q - (2^bits - 1) in {-3..3} or {-7..7}.
+//   bf16: M = 128 (0x4300), fp16: M = 1024 (0x6400).
+template <bool kBf16>
+struct Magic;
+template <>
+struct Magic<true> {
+    static constexpr uint32_t kBits = 0x43004300u;
+    STRATA_DEV static uint32_t sub(uint32_t v, int bits) {
+        // v - (128 + 2^bits - 1) in bf16x2; 131 = 0x4303, 135 = 0x4307
+        __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&v);
+        uint32_t cb = bits == 2 ? 0x43034303u : 0x43074307u;
+        __nv_bfloat162 c = *reinterpret_cast<__nv_bfloat162 *>(&cb);
+        __nv_bfloat162 r = __hsub2(a, c);
+        return *reinterpret_cast<uint32_t *>(&r);
+    }
+};
+template <>
+struct Magic<false> {
+    static constexpr uint32_t kBits = 0x64006400u;
+    STRATA_DEV static uint32_t sub(uint32_t v, int bits) {
+        // v - (1024 + 2^bits - 1) in fp16x2; 1027 = 0x6403, 1031 = 0x6407
+        __half2 a = *reinterpret_cast<__half2 *>(&v);
+        uint32_t cb = bits == 2 ? 0x64036403u : 0x64076407u;
+        __half2 c = *reinterpret_cast<__half2 *>(&cb);
+        __half2 r = __hsub2(a, c);
+        return *reinterpret_cast<uint32_t *>(&r);
+    }
+};
+
+// Register r' (0..7) of block word `lo` (and high-bit word `hi` for 3-bit):
+// a lane pair holding 2q - (2^bits - 1) for the two codes of that register.
+template <bool kBf16, int kBits>
+STRATA_DEV uint32_t dq_pair(uint32_t lo, uint32_t hi, int rp, int hshift) {
+    uint32_t t = rp == 0 ? (lo << 1) : (lo >> (2 * rp - 1));
+    uint32_t v = (t & 0x00060006u) | Magic<kBf16>::kBits;
+    if (kBits == 3) {
+        // high bit of half 0 sits at bit (hshift + rp), of half 1 at bit 16 + hshift + rp;
+        // move both to bit 3 / 19 (the 8s place of 2q).
+        int sh = hshift + rp - 3;
+        uint32_t u = sh >= 0 ? (hi >> sh) : (hi << (-sh));
+        v |= u & 0x00080008u;
+    }
+    return Magic<kBf16>::sub(v, kBits);
+}
+
+}  // namespace strata

@@ -1,0 +1,95 @@
+// Host-side declarations shared by the library's .cu files (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace strata {
+
+// Geometry of one layer on the GPU.
+struct Geometry {
+    int H, E, k, I, Ip, bits;   // Ip: I rounded up to 128 (zero-padded rows / columns)
+    int nseg_h, nseg_i;         // H/128, Ip/128
+    int ub;                     // bytes of one 16x128 unit
+    size_t mat_bytes;           // GPU bytes of one matrix (all three are equal)
+    size_t expert_bytes;        // 3 * mat_bytes
+};
+
+// ---- repack.cu
+// Canonical packed matrix [R][K/32][4*bits] + scales [R][K/32] (device copies)
+// -> GPU layout with Rp rows, Kp columns (zero weights in the padding).
+void launch_repack_matrix(const uint8_t *codes, const uint16_t *scales, int bits, int R, int K,
+                          int Rp, int Kp, uint8_t *out, cudaStream_t s);
+// Debug: dequantise rows [row0, row0+nrows) of a GPU-layout matrix with Kp
+// columns.  kind 0: exact fp32, kind 1: fp16 tensor-core operand (as float).
+void launch_debug_dequant(const uint8_t *mat, int bits, int Kp, int row0, int nrows, int ncols,
+                          int kind, float *out, cudaStream_t s);
+
+// ---- route.cu
+// Router weight in the lane-interleaved layout: Wp[e][H/128][32 lanes][4].
+void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
+                   float *logits, cudaStream_t s);
+void launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                 cudaStream_t s);
+
+// Dispatch scratch for T tokens (chunks of 256 tokens).
+struct DispatchScratch {
+    int32_t *hist;      // [nchunks][E]  per-chunk counts, then per-chunk bases
+    uint32_t *bm;       // [nchunks][8][E] per-warp membership bitmaps
+    int16_t *pre;       // [nchunks][8][E] per-warp exclusive prefix inside the chunk
+};
+size_t dispatch_scratch_bytes(int T, int E);
+void dispatch_scratch_carve(void *base, int T, int E, DispatchScratch *d);
+
+// Units: int4 {expert (E = shared), first slot, n tokens, 0}; tile = tokens per unit.
+// n_units[0] receives the count.  Slots: routed 0..T*k-1 (dispatch order),
+// shared T*k + t.
+int max_units(int T, int k, int E, int tile);
+void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *off,
+                     int32_t *list, int32_t *slot, const DispatchScratch &ds, int4 *units,
+                     int *n_units, int tile, cudaStream_t s);
+
+// ---- gemv.cu (decode)
+struct ExpertWeights {
+    const uint8_t *routed;   // expert e at routed + e * expert_bytes
+    const uint8_t *shared;   // the shared expert
+};
+void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                        const int *n_units, int units_max, const int32_t *list, int Tk,
+                        const void *x, void *a_out, int *err, long long budget, cudaStream_t s);
+void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                      const int *n_units, int units_max, const void *a, float *Y, int *err,
+                      long long budget, cudaStream_t s);
+
+// ---- combine.cu
+// out[t] = Y[Tk + t] + sum_j (ascending expert id) w[t][j] * Y[slot[t][j]]; bf16.
+// y_half: Y stored as fp16 (prefill) instead of fp32 (decode).  residual: h
+// (bf16, in place) <- bf16(f32(h) + f32(bf16(out))) instead of writing out.
+void launch_combine(const void *Y, bool y_half, const int32_t *idx, const float *w,
+                    const int32_t *slot, int T, int k, int H, void *out, bool residual,
+                    cudaStream_t s);
+void launch_rmsnorm(const void *h, void *xn, int T, int H, cudaStream_t s);
+
+// ---- selftest
+void launch_selftest_wait(int *err, long long budget, cudaStream_t s);
+
+// Raise every kernel's dynamic shared-memory limit to the device maximum once
+// per device (outside any stream capture).
+cudaError_t init_kernel_attributes();
+cudaError_t route_init_attributes(int max_smem);
+cudaError_t gemv_init_attributes(int max_smem);
+
+// Allow `f` the largest dynamic shared memory the device permits next to the
+// kernel's static shared memory.
+template <typename F>
+inline cudaError_t allow_max_dyn_smem(F *f, int max_optin) {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(f));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(reinterpret_cast<const void *>(f),
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                max_optin - (int)a.sharedSizeBytes);
+}
+
+}  // namespace strata

@@ -1,0 +1,199 @@
+"""GPU-vs-oracle parity through the C ABI (needs a B200).
+
+Bit-exact: routing indices, per-expert offsets and token lists, dequantised
+weights.  Tolerance (layer specification): bf16 outputs within
+max |err| <= 2e-2 max |ref| and mean relative error <= 5e-3 of the oracle's
+fp64 layer output.  Workloads: the tiny layer (H 256, E 16, k 2, I 64, T 8), the
+Flash-Next-shaped layer (H 2560, E 512, k 10, I 640; the pages' shape: "Strata
+Runs 125B Qwen3.8-Flash-Next on a 12GB Gaming GPU at Up to 94 Tokens/s",
+section "What it is") at decode T = 1, 4 (2-bit), T = 64 (3-bit) and prefill
+T = 8192 (2-bit, sampled outputs), plus ragged and degenerate cases.
+"""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from tests import npref
+from tests.gpu_util import THREADS, W_RTOL, check_output, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import quantized_expert_ffn_04_b200 as qe  # noqa: E402
+
+_layers = {}
+
+
+def layer_of(shape, seed=0, layer=0):
+    key = (shape, seed, layer)
+    if key not in _layers:
+        _layers[key] = gen.layer_weights(shape, seed=seed, layer=layer)
+    return _layers[key]
+
+
+def gpu_layer(shape, T, seed=0, path=0):
+    L = qe.Layer(layer_of(shape, seed), max_tokens=max(T, 1))
+    if path:
+        L.set_option(qe.STRATA_OPT_PATH, path)
+    return L
+
+
+def check_route(L, w, x_bits, T, label):
+    s = w.shape
+    xt = to_dev_bf16(x_bits)
+    idx, wts, off, lst = L.route(xt)
+    L.sync_status()
+    logits = oracle.router_logits(x_bits, w.router_w, w.router_b, threads=THREADS)
+    ridx, rw = oracle.route(logits, s.top_k)
+    cnt, roff, rlst, rslot = oracle.dispatch(ridx, s.n_experts)
+    gi = idx.cpu().numpy()
+    assert np.array_equal(gi, ridx), f"{label}: routing indices differ"
+    np.testing.assert_allclose(wts.cpu().numpy(), rw, rtol=W_RTOL, atol=0)
+    assert np.array_equal(off.cpu().numpy(), roff), f"{label}: offsets differ"
+    assert np.array_equal(lst.cpu().numpy(), rlst), f"{label}: token lists differ"
+    return ridx, roff
+
+
+CASES = [
+    ("tiny", gen.TINY, 8),
+    ("flash2-T1", gen.FLASH2, 1),
+    ("flash2-T4", gen.FLASH2, 4),
+    ("flash2-T13", gen.FLASH2, 13),
+    ("flash3-T64", gen.FLASH3, 64),
+]
+
+
+@pytest.mark.parametrize("name,shape,T", CASES, ids=[c[0] for c in CASES])
+def test_route_and_forward_parity(name, shape, T):
+    w = layer_of(shape)
+    x = gen.hidden(T, shape.hidden, seed=1)
+    L = gpu_layer(shape, T)
+    check_route(L, w, x, T, name)
+    y = from_dev_bf16(L.forward(to_dev_bf16(x)))
+    L.sync_status()
+    _, ref, _, _ = oracle.moe_forward(w, x, threads=THREADS)
+    check_output(y, ref, name)
+
+
+@pytest.mark.parametrize("shape", [gen.TINY, gen.FLASH2, gen.FLASH3], ids=["tiny", "f2", "f3"])
+def test_dequant_bit_exact(shape):
+    w = layer_of(shape)
+    L = gpu_layer(shape, 1)
+    E = shape.n_experts
+    for e in (0, E // 2, E - 1, -1):
+        if e >= 0:
+            ce, se = oracle.expert_slices(shape, w.codes, w.scales, e)
+        else:
+            ce, se = w.shared_codes, w.shared_scales
+        for m in range(3):
+            rows, cols = (shape.inter, shape.hidden) if m < 2 else (shape.hidden, shape.inter)
+            cm, sm = oracle.mat_slices(shape, ce, se, m)
+            r0, nr = (rows // 2 - 8, 24) if rows > 48 else (0, rows)
+            exact = oracle.dequant_rows(cm, sm, shape.bits, cols, r0, nr)
+            got = L.debug_dequant(e, m, r0, nr, kind=0)
+            assert np.array_equal(got.astype(np.float64), exact), (e, m)
+            got16 = L.debug_dequant(e, m, r0, nr, kind=1)
+            assert np.array_equal(got16, exact.astype(np.float16).astype(np.float32)), (e, m)
+
+
+def test_prefill_route_exact_and_sampled_outputs():
+    shape, T = gen.FLASH2, 8192
+    w = layer_of(shape)
+    x = gen.hidden(T, shape.hidden, seed=2)
+    L = gpu_layer(shape, T)
+    ridx, roff = check_route(L, w, x, T, "prefill")
+    y = from_dev_bf16(L.forward(to_dev_bf16(x)))
+    L.sync_status()
+    cnt = np.diff(roff)
+    hot, cold = int(np.argmax(cnt)), int(np.argmin(np.where(cnt > 0, cnt, 1 << 30)))
+    rng = np.random.default_rng(0)
+    sel = set(rng.choice(T, 16, replace=False).tolist()) | {0, T - 1}
+    sel |= set(np.nonzero((ridx == cold).any(axis=1))[0][:4].tolist())
+    sel |= set(np.nonzero((ridx == hot).any(axis=1))[0][:4].tolist())
+    sel = np.array(sorted(sel), dtype=np.int32)
+    _, ref, _, _ = oracle.moe_forward(w, x, sel=sel, threads=THREADS)
+    check_output(y[sel], ref, "prefill sampled")
+    assert np.all(np.isfinite(npref.bf16_bits_to_f64(y)))
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+def test_forced_paths_agree_with_oracle(path):
+    shape, T = gen.FLASH2, 200
+    w = layer_of(shape)
+    x = gen.hidden(T, shape.hidden, seed=3)
+    L = gpu_layer(shape, T, path=path)
+    y = from_dev_bf16(L.forward(to_dev_bf16(x)))
+    L.sync_status()
+    sel = np.arange(0, T, 7, dtype=np.int32)
+    _, ref, _, _ = oracle.moe_forward(w, x, sel=sel, threads=THREADS)
+    check_output(y[sel], ref, f"path {path}")
+
+
+def test_deterministic_across_calls_and_streams():
+    shape, T = gen.FLASH2, 4
+    L = gpu_layer(shape, T)
+    xt = to_dev_bf16(gen.hidden(T, shape.hidden, seed=4))
+    y1 = from_dev_bf16(L.forward(xt))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y2 = L.forward(xt, stream=s)
+    s.synchronize()
+    y3 = from_dev_bf16(L.forward(xt))
+    assert np.array_equal(y1, from_dev_bf16(y2)) and np.array_equal(y1, y3)
+
+
+def test_forward_host_matches_device():
+    shape, T = gen.FLASH2, 4
+    L = gpu_layer(shape, T)
+    x = gen.hidden(T, shape.hidden, seed=5)
+    yd = from_dev_bf16(L.forward(to_dev_bf16(x)))
+    yh = np.empty_like(x)
+    qe.strata_moe_forward_host(L.handle, x.ctypes.data, T, yh.ctypes.data, None)
+    assert np.array_equal(yd, yh)
+
+
+def test_zero_and_oversized_batches():
+    shape = gen.TINY
+    L = gpu_layer(shape, 8)
+    xt = to_dev_bf16(gen.hidden(8, shape.hidden, seed=6))
+    y = torch.zeros_like(xt)
+    qe.strata_moe_forward(L.handle, xt.data_ptr(), 0, y.data_ptr(), None)  # no-op
+    assert int((y.view(torch.int16) != 0).sum()) == 0
+    with pytest.raises(qe.StrataError) as ei:
+        qe.strata_moe_forward(L.handle, xt.data_ptr(), 9, y.data_ptr(), None)
+    assert ei.value.status == qe.STRATA_ERR_INVALID_ARG
+    with pytest.raises(qe.StrataError) as ei:
+        qe.strata_moe_forward(L.handle, xt.data_ptr(), 8, xt.data_ptr() + 64, None)  # overlap
+    assert ei.value.status == qe.STRATA_ERR_INVALID_ARG
+
+
+def test_bounded_waits_report_timeout_and_recover():
+    with pytest.raises(qe.StrataError) as ei:
+        qe.strata_moe_selftest_wait(0, 200000)
+    assert ei.value.status == qe.STRATA_ERR_TIMEOUT
+    shape, T = gen.TINY, 8
+    L = gpu_layer(shape, T)
+    xt = to_dev_bf16(gen.hidden(T, shape.hidden, seed=7))
+    L.set_option(qe.STRATA_OPT_WAIT_BUDGET, 0)
+    L.forward(xt)
+    with pytest.raises(qe.StrataError) as ei:
+        L.sync_status()
+    assert ei.value.status == qe.STRATA_ERR_TIMEOUT
+    L.set_option(qe.STRATA_OPT_WAIT_BUDGET, 4_000_000_000)
+    y = from_dev_bf16(L.forward(xt))
+    L.sync_status()
+    _, ref, _, _ = oracle.moe_forward(layer_of(shape), gen.hidden(T, shape.hidden, seed=7))
+    check_output(y, ref, "after timeout")
+
+
+def test_rmsnorm_bit_exact():
+    x = gen.hidden(37, 2560, seed=8)
+    xt = to_dev_bf16(x)
+    out = torch.empty_like(xt)
+    qe.strata_moe_rmsnorm(xt.data_ptr(), out.data_ptr(), 37, 2560, None)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_bf16(out), oracle.rmsnorm(x))

@@ -1,0 +1,139 @@
+"""Expert-stack parity: h <- h + MoE_l(RMSNorm(h)) over many layers (needs a GPU).
+
+Per layer l the GPU's own layer input h_l (recorded through the stack call's
+trace) is fed to the oracle ("teacher forcing"): RMSNorm must match bit for
+bit, routing indices must match bit for bit, and the layer's residual output
+must stay within the layer tolerance.  Rounding differences compound over
+many layers and can legitimately flip near-ties, so the free-running
+end-to-end result is checked with the same tolerance on the final hidden
+state and the number of routing flips is reported.
+
+Workloads: three tiny layers (T = 8), and the 48-layer Flash-Next-shaped
+stack (48 layers: "Strata Runs 125B Qwen3.8-Flash-Next on a 12GB Gaming GPU at
+Up to 94 Tokens/s", section "What it is"; 512 experts, top-10 + 1 shared,
+I = 640, 2-bit, independent seed per layer) at decode T = 4 and prefill
+T = 8192 (sampled tokens).
+"""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from tests import npref
+from tests.gpu_util import MAX_TOL, MEAN_TOL, THREADS, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import quantized_expert_ffn_04_b200 as qe  # noqa: E402
+
+
+def _ulp_bf16(v):
+    a = np.abs(v)
+    return np.where(a > 0, 2.0 ** (np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7), 2.0 ** -133)
+
+
+def _check_layer_step(h_in, h_out_gpu, layer, sel, label):
+    """Teacher-forced check of one layer on tokens `sel` of the GPU input."""
+    xin = np.ascontiguousarray(h_in[sel])
+    xn = oracle.rmsnorm(xin)
+    yb, yf, ridx, _ = oracle.moe_forward(layer, xn, threads=THREADS)
+    h_ref = oracle.residual_add(xin, yb)
+    got = npref.bf16_bits_to_f64(h_out_gpu[sel])
+    ref = npref.bf16_bits_to_f64(h_ref)
+    # h_out = bf16(h_in + bf16(y)): its error is the layer's output error plus at
+    # most one bf16 rounding of h_out.
+    err = np.maximum(np.abs(got - ref) - _ulp_bf16(ref), 0.0)
+    scale = np.abs(yf)
+    assert err.max() <= MAX_TOL * scale.max(), f"{label}: max err {err.max():.3e}"
+    assert err.sum() <= MEAN_TOL * scale.sum(), f"{label}: mean err {err.sum() / scale.sum():.3e}"
+    return xn, ridx
+
+
+def _gpu_route(handle, xn_bits, k):
+    xt = to_dev_bf16(xn_bits)
+    T = xn_bits.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    qe.strata_moe_route(handle, xt.data_ptr(), T, idx.data_ptr(), w.data_ptr())
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()
+
+
+def _gpu_rmsnorm(h_bits):
+    xt = to_dev_bf16(h_bits)
+    out = torch.empty_like(xt)
+    qe.strata_moe_rmsnorm(xt.data_ptr(), out.data_ptr(), h_bits.shape[0], h_bits.shape[1])
+    torch.cuda.synchronize()
+    return from_dev_bf16(out)
+
+
+def _run_stack(handles, h0_bits):
+    T, H = h0_bits.shape
+    h = to_dev_bf16(h0_bits)
+    trace = torch.empty((len(handles), T, H), dtype=torch.bfloat16, device="cuda")
+    qe.strata_moe_stack_forward(handles, h.data_ptr(), T, trace.data_ptr())
+    qe.strata_moe_sync_status(handles[0])
+    return from_dev_bf16(h), from_dev_bf16(trace)
+
+
+def test_tiny_stack_teacher_forced_and_end_to_end():
+    shape, T, n = gen.TINY, 8, 3
+    layers = [gen.layer_weights(shape, seed=0, layer=l) for l in range(n)]
+    gl = [qe.Layer(w, max_tokens=T) for w in layers]
+    h0 = gen.hidden(T, shape.hidden, seed=0)
+    hf, trace = _run_stack([g.handle for g in gl], h0)
+    sel = np.arange(T)
+    for l in range(n):
+        nxt = trace[l + 1] if l + 1 < n else hf
+        xn, ridx = _check_layer_step(trace[l], nxt, layers[l], sel, f"layer {l}")
+        assert np.array_equal(_gpu_rmsnorm(trace[l]), xn)
+        assert np.array_equal(_gpu_route(gl[l].handle, xn, shape.top_k), ridx)
+    h_ref, _ = oracle.stack_forward(layers, h0)
+    d = np.abs(npref.bf16_bits_to_f64(hf) - npref.bf16_bits_to_f64(h_ref))
+    assert d.max() <= MAX_TOL * np.abs(npref.bf16_bits_to_f64(h_ref)).max()
+
+
+@pytest.fixture(scope="module")
+def flash_stack():
+    shape, n = gen.FLASH2, gen.STACK_LAYERS
+    handles = []
+    for l in range(n):
+        w = gen.layer_weights(shape, seed=0, layer=l)
+        handles.append(qe.Layer(w, max_tokens=8192 if l == 0 else 1))
+        del w
+    yield shape, handles
+    for h in handles:
+        h.close()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T,n_sel", [(4, 4), (8192, 4)], ids=["decode-T4", "prefill-T8192"])
+def test_flash_stack_48_layers(flash_stack, T, n_sel):
+    shape, gl = flash_stack
+    h0 = gen.hidden(T, shape.hidden, seed=11)
+    hf, trace = _run_stack([g.handle for g in gl], h0)
+    sel = np.arange(T) if T == n_sel else np.unique(
+        np.concatenate([[0, T - 1], np.random.default_rng(1).choice(T, n_sel - 2, replace=False)]))
+    n = len(gl)
+    for l in range(n):
+        w = gen.layer_weights(shape, seed=0, layer=l)
+        nxt = trace[l + 1] if l + 1 < n else hf
+        xn, ridx = _check_layer_step(trace[l], nxt, w, sel, f"layer {l}")
+        if l % 8 == 0 or l == n - 1:
+            assert np.array_equal(_gpu_rmsnorm(trace[l][sel]), xn), f"rmsnorm layer {l}"
+            assert np.array_equal(_gpu_route(gl[l].handle, xn, shape.top_k), ridx), \
+                f"routing layer {l}"
+    # free-running end to end on the sampled tokens
+    layers = (gen.layer_weights(shape, seed=0, layer=l) for l in range(n))
+    h = np.ascontiguousarray(h0[sel])
+    for w in layers:
+        yb, _, _, _ = oracle.moe_forward(w, oracle.rmsnorm(h), threads=THREADS)
+        h = oracle.residual_add(h, yb)
+    ref = npref.bf16_bits_to_f64(h)
+    got = npref.bf16_bits_to_f64(hf[sel])
+    rel = np.abs(got - ref).sum() / np.abs(ref).sum()
+    assert rel <= MEAN_TOL, f"end-to-end mean rel err {rel:.3e}"
