@@ -76,6 +76,7 @@ struct strata_moe {
     void *Y = nullptr;            // fp32 (decode) / fp16 (prefill) [slots][H]
     int *err = nullptr;
     void *xio = nullptr, *yio = nullptr, *xn = nullptr;  // bf16 [max_tokens][H]
+    void *x16 = nullptr;                                 // fp16 [max_tokens][H]
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
     // options
     int path = 0;
@@ -156,6 +157,7 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->xio = take(T * H * 2);
     h->yio = take(T * H * 2);
     h->xn = take(T * H * 2);
+    h->x16 = take(T * H * 2);
     return off;
 }
 
@@ -192,7 +194,14 @@ enum { kStRouter, kStTopk, kStDispatch, kStGateUp, kStDown, kStCombine };
 
 void probe(strata_moe_t h, int stage, bool begin, cudaStream_t s) {
     cudaEvent_t e = begin ? h->probe_begin[stage] : h->probe_end[stage];
-    if (e) cudaEventRecord(e, s);
+    if (!e) return;
+    // inside a stream capture the record must become an event node of the graph
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, s);
 }
 
 // Router + top-k + dispatch into the handle's workspace.
@@ -211,23 +220,39 @@ strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStre
     return check_launch("routing kernels");
 }
 
+bool use_decode_path(strata_moe_t h, int T) {
+    if (h->path == 1) return true;
+    if (h->path == 2) return false;
+    return T <= h->decode_max_t;
+}
+
 strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool residual,
                           cudaStream_t s) {
     const Geometry &g = h->geo;
-    strata_status st = run_route(h, x, T, 8, s);
+    const bool decode = use_decode_path(h, T);
+    const int tile = decode ? 8 : kUmmaTile;
+    strata_status st = run_route(h, x, T, tile, s);
     if (st != STRATA_OK) return st;
     ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
-    int umax = max_units(T, g.k, g.E, 8);
-    probe(h, kStGateUp, true, s);
-    launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->a, h->err,
-                       h->budget, s);
-    probe(h, kStGateUp, false, s);
-    probe(h, kStDown, true, s);
-    launch_gemv_down(g, w, h->units, h->n_units, umax, h->a, (float *)h->Y, h->err, h->budget,
-                     s);
-    probe(h, kStDown, false, s);
+    int umax = max_units(T, g.k, g.E, tile);
+    if (decode) {
+        probe(h, kStGateUp, true, s);
+        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->a, h->err,
+                           h->budget, s);
+        probe(h, kStGateUp, false, s);
+        probe(h, kStDown, true, s);
+        launch_gemv_down(g, w, h->units, h->n_units, umax, h->a, (float *)h->Y, h->err,
+                         h->budget, s);
+        probe(h, kStDown, false, s);
+    } else {
+        // the gate/up probe brackets the fp16 token copy, gate/up and down GEMMs
+        probe(h, kStGateUp, true, s);
+        launch_umma_experts(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->x16, h->a,
+                            h->Y, h->err, h->budget, T, s);
+        probe(h, kStGateUp, false, s);
+    }
     probe(h, kStCombine, true, s);
-    launch_combine(h->Y, false, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s);
+    launch_combine(h->Y, !decode, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s);
     probe(h, kStCombine, false, s);
     return check_launch("expert kernels");
 }
@@ -251,7 +276,9 @@ strata_status strata_moe_set_probe(strata_moe_t h, int stage, void *ev_begin, vo
 int strata_moe_launch_count(strata_moe_t h, int T) {
     if (!h || T < 0 || T > h->cfg.max_tokens) return 0;
     if (T == 0) return 0;
-    return 3 /* router, top-k, combine */ + 3 /* dispatch */ + 2 /* gate/up, down */;
+    // router, top-k, 3 dispatch kernels, combine; then gate/up + down, plus the
+    // fp16 token copy on the prefill path
+    return 6 + (use_decode_path(h, T) ? 2 : 3);
 }
 
 strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_weights *wts,

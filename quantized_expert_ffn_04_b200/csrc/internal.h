@@ -62,6 +62,16 @@ void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *uni
                       const int *n_units, int units_max, const void *a, float *Y, int *err,
                       long long budget, cudaStream_t s);
 
+// ---- umma.cu (prefill)
+// x (bf16) -> x16 (fp16 copy), then gate/up (a: fp16 [slots][Ip]) and down
+// (Y: fp16 [slots][H]) on the tensor cores.  Units of up to 256 tokens.
+constexpr int kUmmaTile = 256;
+void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                         const int *n_units, int units_max, const int32_t *list, int Tk,
+                         const void *x, void *x16, void *a, void *Y, int *err, long long budget,
+                         int T, cudaStream_t s);
+cudaError_t umma_init_attributes(int max_smem);
+
 // ---- combine.cu
 // out[t] = Y[Tk + t] + sum_j (ascending expert id) w[t][j] * Y[slot[t][j]]; bf16.
 // y_half: Y stored as fp16 (prefill) instead of fp32 (decode).  residual: h

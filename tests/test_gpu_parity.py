@@ -120,17 +120,39 @@ def test_prefill_route_exact_and_sampled_outputs():
     assert np.all(np.isfinite(npref.bf16_bits_to_f64(y)))
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
-def test_forced_paths_agree_with_oracle(path):
-    shape, T = gen.FLASH2, 200
+PATH_CASES = [
+    ("f2-T200-gemv", gen.FLASH2, 200, 1, 7),
+    ("f2-T200-gemm", gen.FLASH2, 200, 2, 7),
+    ("tiny-T8-gemm", gen.TINY, 8, 2, 1),
+    ("tiny-T300-gemm", gen.TINY, 300, 2, 1),
+    ("f2-T65-auto", gen.FLASH2, 65, 0, 4),
+    ("f3-T160-gemm", gen.FLASH3, 160, 2, 9),
+    ("f3-T64-gemm", gen.FLASH3, 64, 2, 5),
+]
+
+
+@pytest.mark.parametrize("name,shape,T,path,stride", PATH_CASES, ids=[c[0] for c in PATH_CASES])
+def test_paths_agree_with_oracle(name, shape, T, path, stride):
+    """Decode (1) and tensor-core (2) paths at sizes spanning several tiles with a
+    ragged last tile; every `stride`-th token is checked against the oracle."""
     w = layer_of(shape)
     x = gen.hidden(T, shape.hidden, seed=3)
     L = gpu_layer(shape, T, path=path)
     y = from_dev_bf16(L.forward(to_dev_bf16(x)))
     L.sync_status()
-    sel = np.arange(0, T, 7, dtype=np.int32)
+    sel = np.arange(0, T, stride, dtype=np.int32)
     _, ref, _, _ = oracle.moe_forward(w, x, sel=sel, threads=THREADS)
-    check_output(y[sel], ref, f"path {path}")
+    check_output(y[sel], ref, name)
+
+
+def test_paths_agree_with_each_other():
+    """Both paths on the same input: within tolerance of each other, and the
+    routing (shared by both) is identical."""
+    shape, T = gen.FLASH2, 96
+    x = to_dev_bf16(gen.hidden(T, shape.hidden, seed=12))
+    y1 = from_dev_bf16(gpu_layer(shape, T, path=1).forward(x))
+    y2 = from_dev_bf16(gpu_layer(shape, T, path=2).forward(x))
+    check_output(y2, npref.bf16_bits_to_f64(y1), "gemm vs gemv")
 
 
 def test_deterministic_across_calls_and_streams():

@@ -103,7 +103,9 @@ def flash_stack():
     handles = []
     for l in range(n):
         w = gen.layer_weights(shape, seed=0, layer=l)
-        handles.append(qe.Layer(w, max_tokens=8192 if l == 0 else 1))
+        # layer 0's workspace serves the whole stack; the others only route the
+        # few sampled tokens of the per-layer checks
+        handles.append(qe.Layer(w, max_tokens=8192 if l == 0 else 8))
         del w
     yield shape, handles
     for h in handles:
