@@ -198,6 +198,31 @@ strata_status strata_moe_set_probe(strata_moe_t h, int stage, void *ev_begin, vo
 /* Number of kernels one strata_moe_forward of T tokens launches (0 on error). */
 int strata_moe_launch_count(strata_moe_t h, int T);
 
+/* Routing for callers that cannot allocate device memory (code running inside
+ * another framework's memory pool, code on a fixed memory budget, or code that
+ * must not trigger the implicit synchronisation cudaMalloc/cudaFree can cause).
+ * The pages have no counterpart: this is a property of the library, not of the
+ * method.  Same results as strata_moe_route, without a handle:
+ *   x_dev         bf16 [T][H] (device, 16-byte aligned)
+ *   router_w_dev  float [E][H] plain row-major router weight (device)
+ *   router_b_dev  float [E] (device) or NULL for no bias
+ *   idx_dev, w_dev, offsets_dev (or NULL), list_dev (or NULL): as in
+ *                 strata_moe_route
+ * Limits: 1 <= T <= 64 (T == 0 is a no-op), 1 <= E <= 1024,
+ * 1 <= k <= min(E, 32), H a multiple of 128 in [128, 6144]; anything else
+ * returns STRATA_ERR_INVALID_ARG without launching work.
+ * Intermediates live in one static device array of about 0.4 MB that every GPU
+ * loading this library keeps until the process exits; the call allocates
+ * nothing.  The first call on a device looks up that array's device address
+ * (and sets kernel attributes), so make it before any stream capture.  Every
+ * call shares the array, and nothing in it needs to start at zero: each call
+ * overwrites what it reads.  Two calls that overlap on the GPU (different
+ * streams, or different host threads) race on the array. */
+strata_status strata_moe_route_noalloc(const void *x_dev, int T, int H,
+                                       const float *router_w_dev, const float *router_b_dev,
+                                       int E, int k, int32_t *idx_dev, float *w_dev,
+                                       int32_t *offsets_dev, int32_t *list_dev, void *stream);
+
 /* Library version string. */
 const char *strata_moe_version(void);
 

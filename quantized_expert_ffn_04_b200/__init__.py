@@ -30,7 +30,7 @@ SYMBOLS = ("strata_moe_create", "strata_moe_destroy", "strata_moe_route", "strat
            "strata_moe_forward_host", "strata_moe_rmsnorm", "strata_moe_stack_forward",
            "strata_moe_sync_status", "strata_moe_last_error", "strata_moe_debug_dequant",
            "strata_moe_set_option", "strata_moe_selftest_wait", "strata_moe_version",
-           "strata_moe_set_probe", "strata_moe_launch_count")
+           "strata_moe_set_probe", "strata_moe_launch_count", "strata_moe_route_noalloc")
 
 
 class strata_moe_config(C.Structure):
@@ -66,6 +66,7 @@ _sig = {
     "strata_moe_selftest_wait": [_I, _I64],
     "strata_moe_set_probe": [_P, _I, _P, _P],
     "strata_moe_launch_count": [_P, _I],
+    "strata_moe_route_noalloc": [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P],
 }
 for _name, _args in _sig.items():
     _f = getattr(_lib, _name)
@@ -144,6 +145,12 @@ def strata_moe_set_probe(h, stage, ev_begin, ev_end) -> None:
 
 def strata_moe_launch_count(h, T) -> int:
     return _lib.strata_moe_launch_count(h, T)
+
+
+def strata_moe_route_noalloc(x, T, H, router_w, router_b, E, k, idx, w, offsets=None, lst=None,
+                             stream=None) -> None:
+    _check(_lib.strata_moe_route_noalloc(x, T, H, router_w, router_b, E, k, idx, w, offsets, lst,
+                                         stream))
 
 
 # ----------------------------------------------------------------- convenience

@@ -259,6 +259,8 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
 
 }  // namespace
 
+void strata::set_error_message(const char *msg) { g_err = msg; }
+
 extern "C" {
 
 const char *strata_moe_last_error(void) { return g_err.c_str(); }

@@ -84,6 +84,9 @@ void launch_rmsnorm(const void *h, void *xn, int T, int H, cudaStream_t s);
 // ---- selftest
 void launch_selftest_wait(int *err, long long budget, cudaStream_t s);
 
+// Set the thread-local message returned by strata_moe_last_error().
+void set_error_message(const char *msg);
+
 // Raise every kernel's dynamic shared-memory limit to the device maximum once
 // per device (outside any stream capture).
 cudaError_t init_kernel_attributes();
