@@ -129,13 +129,38 @@ def test_flash_stack_48_layers(flash_stack, T, n_sel):
             assert np.array_equal(_gpu_rmsnorm(trace[l][sel]), xn), f"rmsnorm layer {l}"
             assert np.array_equal(_gpu_route(gl[l].handle, xn, shape.top_k), ridx), \
                 f"routing layer {l}"
-    # free-running end to end on the sampled tokens
-    layers = (gen.layer_weights(shape, seed=0, layer=l) for l in range(n))
+    # free-running end to end on the sampled tokens: the oracle follows its own
+    # trajectory; wherever its routing and the GPU's differ, the k-th/(k+1)-th
+    # logit gap must be within the logit perturbation that the accumulated
+    # rounding difference of the two trajectories causes (a near-tie flip).
+    # Tokens that never flip must end within the tolerance.
     h = np.ascontiguousarray(h0[sel])
-    for w in layers:
-        yb, _, _, _ = oracle.moe_forward(w, oracle.rmsnorm(h), threads=THREADS)
+    flipped = np.zeros(len(sel), dtype=bool)
+    report = []
+    k = shape.top_k
+    for l in range(n):
+        w = gen.layer_weights(shape, seed=0, layer=l)
+        xo = oracle.rmsnorm(h)
+        xg = oracle.rmsnorm(np.ascontiguousarray(trace[l][sel]))
+        lo = oracle.router_logits(xo, w.router_w, w.router_b).astype(np.float64)
+        lg = oracle.router_logits(xg, w.router_w, w.router_b).astype(np.float64)
+        io, _ = oracle.route(lo.astype(np.float32), k)
+        ig, _ = oracle.route(lg.astype(np.float32), k)
+        for i in range(len(sel)):
+            if set(io[i]) != set(ig[i]):
+                delta = np.max(np.abs(lo[i] - lg[i]))
+                so, sg = -np.sort(-lo[i]), -np.sort(-lg[i])
+                gap = min(so[k - 1] - so[k], sg[k - 1] - sg[k])
+                report.append((l, int(sel[i]), float(gap), float(delta)))
+                assert gap <= 2 * delta + 1e-6, (
+                    f"layer {l} token {sel[i]}: routing differs with gap {gap:.3e} > "
+                    f"2 x logit perturbation {delta:.3e}")
+                flipped[i] = True
+        yb, _, _, _ = oracle.moe_forward(w, xo, threads=THREADS)
         h = oracle.residual_add(h, yb)
     ref = npref.bf16_bits_to_f64(h)
     got = npref.bf16_bits_to_f64(hf[sel])
-    rel = np.abs(got - ref).sum() / np.abs(ref).sum()
-    assert rel <= MEAN_TOL, f"end-to-end mean rel err {rel:.3e}"
+    print(f"stack T={T}: near-tie routing flips (layer, token, gap, perturbation): {report}")
+    for i in np.nonzero(~flipped)[0]:
+        rel = np.abs(got[i] - ref[i]).sum() / np.abs(ref[i]).sum()
+        assert rel <= MEAN_TOL, f"token {sel[i]} (no routing flip): end-to-end rel err {rel:.3e}"
