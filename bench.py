@@ -49,6 +49,8 @@ WORKLOADS = {
 }
 DEFAULT_WORKLOAD = "decode-t4"
 STAGES = ["router", "topk", "dispatch", "gateup", "down", "combine"]
+TIMING_NOTE = ("CUDA events recorded by the library on the launching stream around the kernel, "
+               "in a second pass of the same graphs and workload right after the timed region")
 GATEUP = 3
 
 
@@ -120,6 +122,21 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ helpers
+def reduce_max(value: float, dist, device) -> float:
+    """Max of `value` over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max / 1000.0)
+
+
 def expert_bytes(shape):
     return shape.expert_bytes
 
@@ -267,29 +284,49 @@ def run_own(args, wl):
         distinct.append(int(torch.unique(idx).numel()))
     torch.cuda.synchronize()
 
-    # ---- probes around the dominant kernel (gate/up), one event pair per layer
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(NL)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(NL)]
-    for e in ev_b + ev_e:
-        e.record(stream)
-    torch.cuda.synchronize()
+    # ---- probes: one CUDA event pair per (layer, stage), recorded by the library
+    # on the launching stream around each stage.  They are captured into a
+    # second set of graphs used only for the per-stage pass: event nodes between
+    # kernels would also cut the programmatic-launch chain of the headline steps.
+    decode = T <= 64
+    stages = ([0, 1] if T <= 256 else [0, 2]) + [3, 4, 5]
+    ev_b = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(NL)]
+    ev_e = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(NL)]
     for l in range(NL):
-        qe.strata_moe_set_probe(layers[l].handle, GATEUP, ev_b[l].cuda_event, ev_e[l].cuda_event)
+        for st in stages:
+            ev_b[l][st].record(stream)
+            ev_e[l][st].record(stream)
+    torch.cuda.synchronize()
 
-    # ---- warm-up eagerly, then capture one graph per layer
+    def set_probes(on: bool):
+        for l in range(NL):
+            for st in stages:
+                qe.strata_moe_set_probe(layers[l].handle, st,
+                                        ev_b[l][st].cuda_event if on else None,
+                                        ev_e[l][st].cuda_event if on else None)
+
+    # ---- warm-up eagerly, then capture one graph per layer (plain and probed)
     for l in range(NL):
         layers[l].forward(xs[l], out=ys[l], stream=stream)
     torch.cuda.synchronize()
     for l in range(NL):
         layers[l].sync_status(stream)
-    graphs = []
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
-    for l in range(NL):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            layers[l].forward(xs[l], out=ys[l], stream=cap)
-        graphs.append(g)
+
+    def capture():
+        gs = []
+        for l in range(NL):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                layers[l].forward(xs[l], out=ys[l], stream=cap)
+            gs.append(g)
+        return gs
+
+    graphs = capture()
+    set_probes(True)
+    graphs_probe = capture()
+    set_probes(False)
     stream.wait_stream(cap)
     torch.cuda.synchronize()
     for i in range(args.warmup):
@@ -311,29 +348,52 @@ def run_own(args, wl):
     ms = t_start.elapsed_time(t_end)
     for l in range(NL):
         layers[l].sync_status(stream)
-    # dominant kernel: the last launch of each layer's graph inside the region
-    ran = sorted({i % NL for i in range(max(0, args.steps - NL), args.steps)})
-    gu_ms = [ev_b[l].elapsed_time(ev_e[l]) for l in ran]
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, dist, "cuda")
     ms_step = ms / args.steps
-    tokens = T * args.steps * world
-    value = tokens / (ms / 1000.0)
+    value = weak_scaling_value(T * args.steps, world, ms)
 
-    # ---- algorithmic bytes
-    mb = mat_bytes(shape)
-    gu_bytes = [(distinct[l] + 1) * 2 * mb + T * shape.hidden * 2 for l in ran]
-    achieved = sum(gu_bytes) / (sum(gu_ms) / 1000.0) / 1e9  # GB/s
-    peak = float(peaks["hbm_gbs"])
+    # ---- per-stage pass: the probed graphs, same workload; each layer's event
+    # pairs hold its last launch
+    probe_steps = max(NL, min(args.steps, 200))
+    for i in range(probe_steps):
+        graphs_probe[i % NL].replay()
+    torch.cuda.synchronize()
+    for l in range(NL):
+        layers[l].sync_status(stream)
+    ran = list(range(NL))
+    stage_ms = {STAGES[st]: statistics.mean(ev_b[l][st].elapsed_time(ev_e[l][st]) for l in ran)
+                for st in stages}
+    if T <= 256:
+        stage_ms["topk+dispatch"] = stage_ms.pop("topk")
+
+    # ---- roofline of the dominant kernel (gate/up + SwiGLU)
+    gu_ms = statistics.mean(ev_b[l][GATEUP].elapsed_time(ev_e[l][GATEUP]) for l in ran)
+    if decode:
+        mb = mat_bytes(shape)
+        gu_work = statistics.mean((distinct[l] + 1) * 2 * mb + T * shape.hidden * 2 for l in ran)
+        achieved = gu_work / (gu_ms / 1000.0) / 1e9  # GB/s
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "kernel": "gemv_gateup", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind + " hbm copy",
+                "traffic": traffic_from_profile(wl), "algorithmic_bytes_per_launch": gu_work,
+                "launch_ms": gu_ms, "timing": TIMING_NOTE}
+    else:
+        pairs = T * (shape.top_k + 1)
+        ip = (shape.inter + 127) // 128 * 128
+        gu_work = 2.0 * 2 * shape.hidden * ip * pairs  # gate + up, 2 flops per MAC
+        achieved = gu_work / (gu_ms / 1000.0) / 1e12  # TFLOP/s
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roof = {"bound": "tensor", "kernel": "umma_expert_kernel (gate/up, fp16 operands)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": peak_kind + " bf16 sustained (fp16 runs at the bf16 rate)",
+                "traffic": traffic_from_profile(wl), "algorithmic_flops_per_launch": gu_work,
+                "launch_ms": gu_ms, "timing": TIMING_NOTE}
     step_bytes = [shape.n_experts * shape.hidden * 4 + shape.n_experts * 4
                   + (distinct[l] + 1) * shape.expert_bytes + 2 * T * shape.hidden * 2
                   for l in range(NL)]
+    step_flops = 2.0 * 3 * shape.hidden * shape.inter * T * (shape.top_k + 1)
 
     # ---- e2e through the host-buffer entry point (pinned host memory)
-    for l in range(NL):
-        qe.strata_moe_set_probe(layers[l].handle, GATEUP, None, None)
     xh = [torch.from_numpy(x.view(np.int16).copy()).pin_memory() for x in xs_host]
     yh = [torch.empty_like(x).pin_memory() for x in xh]
     e2e_steps = min(args.steps, args.e2e_steps)
@@ -352,12 +412,8 @@ def run_own(args, wl):
                                    stream.cuda_stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = T * e2e_steps * world / (e2e_ms / 1000.0)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dist, "cuda")
+    e2e_value = weak_scaling_value(T * e2e_steps, world, e2e_ms)
 
     # ---- CPU baseline (rank 0, N = 1 only)
     cpu = None
@@ -383,14 +439,12 @@ def run_own(args, wl):
                          "expert weights)" % (NL, NL * (shape.n_experts + 1)
                                               * shape.expert_bytes / 1e9),
                    "cuda_graphs": True, "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_gateup", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind,
-                     "traffic": traffic_from_profile(wl),
-                     "algorithmic_bytes_per_launch": statistics.mean(gu_bytes),
-                     "launch_ms": statistics.mean(gu_ms)},
+        "roofline": roof,
+        "stages_ms": stage_ms,
         "step_bytes": statistics.mean(step_bytes),
-        "step_hbm_frac": statistics.mean(step_bytes) / (ms_step / 1000.0) / 1e9 / peak,
+        "step_hbm_frac": statistics.mean(step_bytes) / (ms_step / 1000.0) / 1e9
+                         / float(peaks["hbm_gbs"]),
+        "step_tflops": step_flops / (ms_step / 1000.0) / 1e12,
         "distinct_experts": statistics.mean(distinct),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
@@ -400,9 +454,8 @@ def run_own(args, wl):
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                    "reasons": clk["reasons"], "samples": clk["samples"]},
     }
-    for g in graphs:
-        del g
     graphs.clear()
+    graphs_probe.clear()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

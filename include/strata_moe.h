@@ -188,8 +188,11 @@ strata_status strata_moe_selftest_wait(int device, int64_t budget_cycles);
 
 /* Profiling hook: make every later forward of `h` record CUDA event
  * `ev_begin` (a cudaEvent_t passed as void*) on the call's stream just before
- * the kernel(s) of `stage` and `ev_end` just after them.  Stages: 0 router,
- * 1 top-k, 2 dispatch, 3 gate/up + SwiGLU, 4 down, 5 combine.  NULL events
+ * the kernel(s) of `stage` and `ev_end` just after them.  Stages: 0 router
+ * (for T > 256: the fp16 token copy, the screening GEMM and the screened
+ * top-k), 1 top-k + dispatch (T <= 256, one kernel), 2 dispatch (T > 256),
+ * 3 gate/up + SwiGLU (on the prefill path with T <= 256 also the fp16 token
+ * copy), 4 down, 5 combine.  NULL events
  * switch the probe off.  The events must be created by the caller on the
  * handle's device (with timing enabled); forwards captured into a CUDA graph
  * capture the event records too. */

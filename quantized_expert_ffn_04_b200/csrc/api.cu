@@ -8,6 +8,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
+#include <cmath>
 #include <string>
 #include <vector>
 
@@ -63,6 +65,9 @@ struct strata_moe {
     uint8_t *wq = nullptr;        // (E + 1) experts; the shared expert last
     float *router_wp = nullptr;   // [E][H/128][32][4]
     float *router_b = nullptr;    // [E] or null
+    __half *router_split = nullptr;  // [router_rows][H]: fp16(W) rows, then fp16(W - fp16(W))
+    int router_rows = 0;             // 2E rounded up to 128
+    float screen_gam = 0.f, screen_wmax = 0.f, screen_bmax = 0.f;
     void *ws = nullptr;
     size_t ws_bytes = 0;
     // workspace views
@@ -77,6 +82,7 @@ struct strata_moe {
     int *err = nullptr;
     void *xio = nullptr, *yio = nullptr, *xn = nullptr;  // bf16 [max_tokens][H]
     void *x16 = nullptr;                                 // fp16 [max_tokens][H]
+    float *dsplit = nullptr;  // [max_tokens][router_rows] screening GEMM output (T > 256)
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
     // options
     int path = 0;
@@ -158,6 +164,7 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->yio = take(T * H * 2);
     h->xn = take(T * H * 2);
     h->x16 = take(T * H * 2);
+    h->dsplit = (float *)take(T > (size_t)kSmallMaxT ? T * (size_t)h->router_rows * 4 : 0);
     return off;
 }
 
@@ -166,6 +173,7 @@ void free_handle(strata_moe *h) {
     cudaFree(h->wq);
     cudaFree(h->router_wp);
     cudaFree(h->router_b);
+    cudaFree(h->router_split);
     cudaFree(h->ws);
     delete h;
 }
@@ -204,19 +212,35 @@ void probe(strata_moe_t h, int stage, bool begin, cudaStream_t s) {
         cudaEventRecord(e, s);
 }
 
-// Router + top-k + dispatch into the handle's workspace.
+// Router + top-k + dispatch into the handle's workspace.  Above kSmallMaxT
+// tokens the router runs on the tensor cores (screening GEMM on the fp16 copy
+// of x, which the prefill experts reuse) followed by the exact recompute of
+// the candidates.
 strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStream_t s) {
     const Geometry &g = h->geo;
     probe(h, kStRouter, true, s);
-    launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s);
+    if (T > kSmallMaxT) {
+        launch_to_half(x, h->x16, (size_t)T * g.H, s);
+        launch_umma_plain(h->router_split, h->router_rows, (const __half *)h->x16, T, g.H,
+                          h->dsplit, h->err, h->budget, s);
+        launch_screen_topk(h->dsplit, h->router_rows, x, T, g.H, h->router_wp, h->router_b, g.E,
+                           g.k, h->screen_gam, h->screen_wmax, h->screen_bmax, h->idx, h->wts, s);
+    } else {
+        launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s);
+    }
     probe(h, kStRouter, false, s);
-    probe(h, kStTopk, true, s);
-    launch_topk(h->logits, T, g.E, g.k, h->idx, h->wts, s);
-    probe(h, kStTopk, false, s);
-    probe(h, kStDispatch, true, s);
-    launch_dispatch(h->idx, T, g.k, g.E, h->cnt, h->off, h->list, h->slot, h->ds, h->units,
-                    h->n_units, tile, s);
-    probe(h, kStDispatch, false, s);
+    if (T > kSmallMaxT) {
+        probe(h, kStDispatch, true, s);
+        launch_dispatch(h->idx, T, g.k, g.E, h->cnt, h->off, h->list, h->slot, h->ds, h->units,
+                        h->n_units, tile, s);
+        probe(h, kStDispatch, false, s);
+    } else {
+        // top-k and dispatch fused in one CTA (the top-k probe brackets both)
+        probe(h, kStTopk, true, s);
+        launch_route_small(h->logits, T, g.E, g.k, h->idx, h->wts, h->cnt, h->off, h->list,
+                           h->slot, h->units, h->n_units, tile, s);
+        probe(h, kStTopk, false, s);
+    }
     return check_launch("routing kernels");
 }
 
@@ -237,19 +261,24 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
     int umax = max_units(T, g.k, g.E, tile);
     if (decode) {
         probe(h, kStGateUp, true, s);
-        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->a, h->err,
-                           h->budget, s);
+        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, T, x, h->a,
+                           h->err, h->budget, s);
         probe(h, kStGateUp, false, s);
         probe(h, kStDown, true, s);
-        launch_gemv_down(g, w, h->units, h->n_units, umax, h->a, (float *)h->Y, h->err,
+        launch_gemv_down(g, w, h->units, h->n_units, umax, T, h->a, (float *)h->Y, h->err,
                          h->budget, s);
         probe(h, kStDown, false, s);
     } else {
-        // the gate/up probe brackets the fp16 token copy, gate/up and down GEMMs
+        // the gate/up probe brackets the gate/up GEMM (and, for T <= kSmallMaxT,
+        // the fp16 token copy, which larger batches make in the router stage)
         probe(h, kStGateUp, true, s);
-        launch_umma_experts(g, w, h->units, h->n_units, umax, h->list, T * g.k, x, h->x16, h->a,
-                            h->Y, h->err, h->budget, T, s);
+        if (T <= kSmallMaxT) launch_to_half(x, h->x16, (size_t)T * g.H, s);
+        launch_umma_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, h->x16, h->a,
+                           h->err, h->budget, s);
         probe(h, kStGateUp, false, s);
+        probe(h, kStDown, true, s);
+        launch_umma_down(g, w, h->units, h->n_units, umax, h->a, h->Y, h->err, h->budget, s);
+        probe(h, kStDown, false, s);
     }
     probe(h, kStCombine, true, s);
     launch_combine(h->Y, !decode, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s);
@@ -278,9 +307,13 @@ strata_status strata_moe_set_probe(strata_moe_t h, int stage, void *ev_begin, vo
 int strata_moe_launch_count(strata_moe_t h, int T) {
     if (!h || T < 0 || T > h->cfg.max_tokens) return 0;
     if (T == 0) return 0;
-    // router, top-k, 3 dispatch kernels, combine; then gate/up + down, plus the
-    // fp16 token copy on the prefill path
-    return 6 + (use_decode_path(h, T) ? 2 : 3);
+    // up to kSmallMaxT tokens: router, fused top-k + dispatch; above: fp16 token
+    // copy, screening GEMM, screened top-k, 3 dispatch kernels.  Then gate/up +
+    // down (+ the fp16 token copy on the prefill path when T <= kSmallMaxT),
+    // and the combine.
+    const bool decode = use_decode_path(h, T);
+    if (T <= kSmallMaxT) return 2 + (decode ? 2 : 3) + 1;
+    return 6 + 2 + 1;
 }
 
 strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_weights *wts,
@@ -306,6 +339,7 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
     h->device = device;
     h->cfg = *cfg;
     h->geo = make_geometry(*cfg);
+    h->router_rows = (2 * cfg->n_experts + 127) / 128 * 128;
     const Geometry &g = h->geo;
     const size_t H = g.H, E = g.E;
 
@@ -337,6 +371,34 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
                 wp[((e * (H / 128) + s4) * 32 + l) * 4 + j] = wts->router_w[e * H + i];
             }
         ce = cudaMemcpy(h->router_wp, wp.data(), E * H * 4, cudaMemcpyHostToDevice);
+        // screening split W = fp16(W) + fp16(W - fp16(W)) and the bound's constants
+        const size_t R = (size_t)h->router_rows;
+        std::vector<__half> split(R * H, __float2half_rn(0.0f));
+        double wmax = 0.0, bmax = 0.0;
+        for (size_t e = 0; e < E; e++) {
+            double n2 = 0.0;
+            for (size_t i = 0; i < H; i++) {
+                float w = wts->router_w[e * H + i];
+                __half hi = __float2half_rn(w);
+                split[e * H + i] = hi;
+                split[(E + e) * H + i] = __float2half_rn(w - __half2float(hi));
+                n2 += (double)w * w;
+            }
+            wmax = std::max(wmax, std::sqrt(n2));
+            if (cfg->has_router_bias) bmax = std::max(bmax, (double)std::fabs(wts->router_b[e]));
+        }
+        h->screen_wmax = (float)(wmax * (1.0 + 1e-6));
+        h->screen_bmax = (float)(bmax * (1.0 + 1e-6));
+        h->screen_gam = (float)(H * std::ldexp(1.0, -23) + std::ldexp(1.0, -22) +
+                                (H / 32.0 + 10.0) * std::ldexp(1.0, -24));
+        if (ce == cudaSuccess) {
+            if (cudaMalloc(&h->router_split, R * H * 2) != cudaSuccess) {
+                cudaGetLastError();
+                free_handle(h);
+                return fail(STRATA_ERR_OOM, "router split allocation failed");
+            }
+            ce = cudaMemcpy(h->router_split, split.data(), R * H * 2, cudaMemcpyHostToDevice);
+        }
         if (ce == cudaSuccess && cfg->has_router_bias)
             ce = cudaMemcpy(h->router_b, wts->router_b, E * 4, cudaMemcpyHostToDevice);
         if (ce != cudaSuccess) {
@@ -534,11 +596,16 @@ strata_status strata_moe_stack_forward(const strata_moe_t *layers, int n_layers,
             if (ce != cudaSuccess) return cuda_fail(ce, "trace copy");
         }
         launch_rmsnorm(h_dev, l0->xn, T, l0->geo.H, s);
-        // run layer L's weights in layer 0's workspace
+        // run layer L's weights (everything create() derived from them) in
+        // layer 0's workspace
         strata_moe view = *l0;
         view.wq = L->wq;
         view.router_wp = L->router_wp;
         view.router_b = L->router_b;
+        view.router_split = L->router_split;
+        view.screen_gam = L->screen_gam;
+        view.screen_wmax = L->screen_wmax;
+        view.screen_bmax = L->screen_bmax;
         view.cfg.has_router_bias = L->cfg.has_router_bias;
         st = run_forward(&view, l0->xn, T, h_dev, true, s);
         if (st != STRATA_OK) return st;

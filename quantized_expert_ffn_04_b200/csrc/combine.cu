@@ -14,84 +14,97 @@
 
 namespace strata {
 
+// 8 consecutive columns of a staging row as fp32.
 template <typename YT>
-__device__ __forceinline__ float4 load4(const YT *p);
+__device__ __forceinline__ void load8(const YT *p, float (&v)[8]);
 template <>
-__device__ __forceinline__ float4 load4<float>(const float *p) {
-    return *reinterpret_cast<const float4 *>(p);
+__device__ __forceinline__ void load8<float>(const float *p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4 *>(p);
+    float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
 }
 template <>
-__device__ __forceinline__ float4 load4<__half>(const __half *p) {
-    uint2 v = *reinterpret_cast<const uint2 *>(p);
-    float2 a = __half22float2(*reinterpret_cast<__half2 *>(&v.x));
-    float2 b = __half22float2(*reinterpret_cast<__half2 *>(&v.y));
-    return make_float4(a.x, a.y, b.x, b.y);
+__device__ __forceinline__ void load8<__half>(const __half *p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
 }
 
+// grid: (T, column blocks of 512); 64 threads x 8 columns.  The k picks of the
+// token are read in parallel and placed by rank of their expert id (ids of one
+// token are distinct), then summed in that order.
+constexpr int kCombineCols = 512;
+constexpr int kCombineThreads = 64;
+
 template <typename YT>
-__global__ __launch_bounds__(256) void combine_kernel(const YT *__restrict__ Y,
-                                                      const int32_t *__restrict__ idx,
-                                                      const float *__restrict__ w,
-                                                      const int32_t *__restrict__ slot, int T,
-                                                      int k, int H, __nv_bfloat16 *out,
-                                                      int residual) {
-    __shared__ int se[32], ss[32];
-    __shared__ float sw[32];
+__global__ __launch_bounds__(kCombineThreads) void combine_kernel(
+    const YT *__restrict__ Y, const int32_t *__restrict__ idx, const float *__restrict__ w,
+    const int32_t *__restrict__ slot, int T, int k, int H, __nv_bfloat16 *out, int residual) {
+    __shared__ int re[32], rs[32], ss[32];
+    __shared__ float rw[32], sw[32];
     const int t = blockIdx.x;
-    if (threadIdx.x == 0) {
-        // insertion sort of the k picks by expert id
-        for (int j = 0; j < k; j++) {
-            int e = idx[(size_t)t * k + j], s = slot[(size_t)t * k + j];
-            float wj = w[(size_t)t * k + j];
-            int p = j;
-            while (p > 0 && se[p - 1] > e) {
-                se[p] = se[p - 1];
-                ss[p] = ss[p - 1];
-                sw[p] = sw[p - 1];
-                p--;
-            }
-            se[p] = e;
-            ss[p] = s;
-            sw[p] = wj;
-        }
+    const int j = threadIdx.x;
+    // the picks come from routing, long finished; the expert outputs need the
+    // previous kernel
+    if (j < k) {
+        re[j] = __ldcg(idx + (size_t)t * k + j);
+        rs[j] = __ldcg(slot + (size_t)t * k + j);
+        rw[j] = __ldcg(w + (size_t)t * k + j);
+    }
+    grid_dependency_wait();
+    __syncthreads();
+    if (j < k) {
+        int rank = 0;
+        for (int i = 0; i < k; i++) rank += re[i] < re[j];
+        ss[rank] = rs[j];
+        sw[rank] = rw[j];
     }
     __syncthreads();
     const size_t Tk = (size_t)T * k;
-    for (int c = threadIdx.x * 4; c < H; c += blockDim.x * 4) {
-        float4 acc = load4<YT>(Y + (Tk + t) * H + c);
-        for (int j = 0; j < k; j++) {
-            float4 v = load4<YT>(Y + (size_t)ss[j] * H + c);
-            float wj = sw[j];
-            acc.x = fmaf(wj, v.x, acc.x);
-            acc.y = fmaf(wj, v.y, acc.y);
-            acc.z = fmaf(wj, v.z, acc.z);
-            acc.w = fmaf(wj, v.w, acc.w);
-        }
-        __nv_bfloat16 *o = out + (size_t)t * H + c;
-        float r[4] = {acc.x, acc.y, acc.z, acc.w};
-        __nv_bfloat16 ob[4];
+    const int c = blockIdx.y * kCombineCols + threadIdx.x * 8;
+    if (c >= H) return;
+    float acc[8];
+    load8<YT>(Y + (Tk + t) * H + c, acc);
+#pragma unroll 4
+    for (int i = 0; i < k; i++) {
+        float v[8];
+        load8<YT>(Y + (size_t)ss[i] * H + c, v);
+        const float wi = sw[i];
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            __nv_bfloat16 yb = __float2bfloat16_rn(r[i]);
-            if (residual)
-                ob[i] = __float2bfloat16_rn(__fadd_rn(__bfloat162float(o[i]), __bfloat162float(yb)));
-            else
-                ob[i] = yb;
-        }
-        *reinterpret_cast<uint2 *>(o) = *reinterpret_cast<uint2 *>(ob);
+        for (int q = 0; q < 8; q++) acc[q] = fmaf(wi, v[q], acc[q]);
     }
+    __nv_bfloat16 *o = out + (size_t)t * H + c;
+    uint4 hv = make_uint4(0, 0, 0, 0);
+    if (residual) hv = *reinterpret_cast<const uint4 *>(o);
+    const __nv_bfloat16 *hb = reinterpret_cast<const __nv_bfloat16 *>(&hv);
+    __nv_bfloat16 ob[8];
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+        __nv_bfloat16 yb = __float2bfloat16_rn(acc[q]);
+        ob[q] = residual ? __float2bfloat16_rn(__fadd_rn(__bfloat162float(hb[q]), __bfloat162float(yb)))
+                         : yb;
+    }
+    *reinterpret_cast<uint4 *>(o) = *reinterpret_cast<uint4 *>(ob);
 }
 
 void launch_combine(const void *Y, bool y_half, const int32_t *idx, const float *w,
                     const int32_t *slot, int T, int k, int H, void *out, bool residual,
                     cudaStream_t s) {
     auto o = reinterpret_cast<__nv_bfloat16 *>(out);
+    dim3 grid(T, (H + kCombineCols - 1) / kCombineCols);
     if (y_half)
-        combine_kernel<__half><<<T, 256, 0, s>>>(reinterpret_cast<const __half *>(Y), idx, w, slot,
-                                                 T, k, H, o, residual ? 1 : 0);
+        launch_pdl(combine_kernel<__half>, grid, dim3(kCombineThreads), 0, s,
+                   reinterpret_cast<const __half *>(Y), idx, w, slot, T, k, H, o,
+                   residual ? 1 : 0);
     else
-        combine_kernel<float><<<T, 256, 0, s>>>(reinterpret_cast<const float *>(Y), idx, w, slot,
-                                                T, k, H, o, residual ? 1 : 0);
+        launch_pdl(combine_kernel<float>, grid, dim3(kCombineThreads), 0, s,
+                   reinterpret_cast<const float *>(Y), idx, w, slot, T, k, H, o,
+                   residual ? 1 : 0);
 }
 
 // ------------------------------------------------------------------ RMSNorm

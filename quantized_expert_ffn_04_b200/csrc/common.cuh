@@ -18,8 +18,13 @@ namespace strata {
 //                     lane L = 4g + c owns 16 bytes = 4 words, word w = block w
 //                     of the segment (32 columns).  Bit positions inside word w
 //                     for fragment register r' = 4s + r (s = k-step of the block,
-//                     r = mma A register 0..3): half 0 at bits 2r'..2r'+1,
-//                     half 1 at bits 16+2r'..16+2r'+1.
+//                     r = mma A register 0..3): half 0 at bits P..P+1, half 1 at
+//                     bits 16+P..16+P+1, with P = code_pos(bits, r'):
+//                       2-bit: P = 2, 4, 6, 8, 10, 12, 14, 0 for r' = 0..7, so
+//                              that r' = 0..3 come out of one mask (the code sits
+//                              in the fp16 mantissa at bit 2, 4, 6 or 8), r' = 4..6
+//                              after one shift by 8 and r' = 7 after a shift by 2;
+//                       3-bit: P = 2r'.
 //                     Register r holds (row, col) pairs of the m16n8k16 A
 //                     fragment: r=0 (g, 2c|2c+1), r=1 (g+8, 2c|2c+1),
 //                     r=2 (g, 2c+8|2c+9), r=3 (g+8, 2c+8|2c+9); col relative to
@@ -33,6 +38,10 @@ constexpr int kSegCols = 128;
 constexpr int kLoBytes = 512;
 constexpr int kHiBytes = 256;
 constexpr int kScaleBytes = 128;
+
+__host__ __device__ constexpr int code_pos(int bits, int rp) {
+    return bits == 2 ? (rp < 7 ? 2 * rp + 2 : 0) : 2 * rp;
+}
 
 __host__ __device__ constexpr int unit_bytes(int bits) {
     return kLoBytes + (bits == 3 ? kHiBytes : 0) + kScaleBytes;
@@ -82,6 +91,21 @@ STRATA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep in hardware for up to `hint_ns`
+// nanoseconds waiting for the phase (instead of spinning on issue slots).
+STRATA_DEV bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kSleepHintNs = 100000;  // re-check the wait budget every 0.1 ms
+
 // Wait for phase `parity` of `bar`, giving up after `budget` SM cycles.  On
 // give-up the handle's error word gets kErrTimeout and false is returned.
 STRATA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget, int *err) {
@@ -90,7 +114,7 @@ STRATA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget, int 
         return false;
     }
     long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
         if (clock64() - t0 > budget) {
             if (err) atomicCAS(err, 0, kErrTimeout);
             return false;
@@ -117,6 +141,16 @@ STRATA_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *b
             "r"(smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Programmatic dependent launch: block until the preceding kernel in the
+// stream has completed and its memory is visible (a no-op when the kernel was
+// launched without the programmatic-serialization attribute).
+STRATA_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel of the stream start launching once every CTA of this
+// grid has called this (or exited).
+STRATA_DEV void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 STRATA_DEV void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
@@ -289,6 +323,76 @@ STRATA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "m
 template <int N>
 STRATA_DEV void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace strata
+
+// ---------------------------------------------------------------- 2-bit fast path
+namespace strata {
+
+// A code q at mantissa bit pe of the fp16 value M = 1024 (0x6400, ulp 1) gives
+// h = 1024 + q 2^pe exactly; fma(h, 2^(1-pe), -(1024 2^(1-pe) + 3)) is the
+// exact small integer 2q - 3 (one rounding of an exact value).  Multipliers
+// and offsets for pe = 2, 4, 6, 8 as fp16 pairs:
+STRATA_DEV uint32_t dq2_mul(int j) {
+    return j == 0 ? 0x38003800u : j == 1 ? 0x30003000u : j == 2 ? 0x28002800u : 0x20002000u;
+}
+STRATA_DEV uint32_t dq2_off(int j) {
+    return j == 0 ? 0xE006E006u : j == 1 ? 0xD818D818u : j == 2 ? 0xD060D060u : 0xC980C980u;
+}
+
+STRATA_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Register r' (0..7) of a 2-bit block word: fp16 pair of 2q - 3.
+STRATA_DEV uint32_t dq2_pair(uint32_t w, int rp) {
+    const uint32_t src = rp < 4 ? w : (rp < 7 ? (w >> 8) : (w << 2));
+    const int j = rp < 4 ? rp : (rp < 7 ? rp - 4 : 0);  // pe = 2 j + 2
+    const uint32_t mask = (3u << (2 * j + 2)) | (3u << (16 + 2 * j + 2));
+    return hfma2_u32((src & mask) | 0x64006400u, dq2_mul(j), dq2_off(j));
+}
+
+// One 32-wide block of a 2-bit matrix against 8 token columns, fp16
+// operands, fp32 result d (fresh): the 8 fragment registers are extracted from
+// word w (2 shifts, 8 mask/or, 8 packed fma) and fed to two m16n8k16 mma in
+// one asm block so they land directly in the operand registers.
+STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, uint32_t b2,
+                           uint32_t b3) {
+    asm volatile(
+        "{\n\t"
+        ".reg .b32 s8, s2, h0, h1, h2, h3, h4, h5, h6, h7;\n\t"
+        ".reg .f32 z;\n\t"
+        "mov.f32 z, 0f00000000;\n\t"
+        "shr.b32 s8, %4, 8;\n\t"
+        "shl.b32 s2, %4, 2;\n\t"
+        "lop3.b32 h0, %4, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h1, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h2, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h3, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h4, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h5, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h6, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h7, s2, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "fma.rn.f16x2 h0, h0, %9, %13;\n\t"
+        "fma.rn.f16x2 h1, h1, %10, %14;\n\t"
+        "fma.rn.f16x2 h2, h2, %11, %15;\n\t"
+        "fma.rn.f16x2 h3, h3, %12, %16;\n\t"
+        "fma.rn.f16x2 h4, h4, %9, %13;\n\t"
+        "fma.rn.f16x2 h5, h5, %10, %14;\n\t"
+        "fma.rn.f16x2 h6, h6, %11, %15;\n\t"
+        "fma.rn.f16x2 h7, h7, %9, %13;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h0,h1,h2,h3}, "
+        "{%5,%6}, {z,z,z,z};\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h4,h5,h6,h7}, "
+        "{%7,%8}, {%0,%1,%2,%3};\n\t"
+        "}\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(0x38003800u), "r"(0x30003000u),
+          "r"(0x28002800u), "r"(0x20002000u), "r"(0xE006E006u), "r"(0xD818D818u),
+          "r"(0xD060D060u), "r"(0xC980C980u));
 }
 
 }  // namespace strata

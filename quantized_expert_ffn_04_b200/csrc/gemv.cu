@@ -13,11 +13,14 @@
 // are all issued at kernel start, so every byte the CTA needs is in flight at
 // once.  The codes are turned into exact small odd integers 2q-(2^bits-1) in
 // registers (two per 32-bit lane pair: shift, mask/or against a magic
-// exponent, one packed subtract), the tensor core reduces 16x16 blocks against
-// the staged token rows (mma.sync m16n8k16, fp32 accumulate), and each 32-wide
-// block's partial is scaled by its fp16 scale in fp32.  The tensor core is
-// used only as the in-warp reduction: products are exact (small integer x
-// bf16/fp16), so the result is the exact dot product up to fp32 rounding.
+// exponent, one packed fp16 subtract), the tensor core reduces 16x16 blocks
+// against the staged token rows (mma.sync m16n8k16, fp16 operands, fp32
+// accumulate), and each 32-wide block's partial is scaled by its fp16 scale in
+// fp32.  The tensor core is used only as the in-warp reduction: products are
+// exact (small integer x fp16), so the result is the dot product up to fp32
+// rounding.  Token rows (bf16) are staged as fp16, which holds every bf16
+// value of magnitude 2^-14 .. 65504 exactly; only as many rows are staged as
+// the batch can put in one unit, so small batches fit more CTAs per SM.
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,26 +34,28 @@ __device__ __forceinline__ uint32_t comp4(const uint4 &v, int i) {
 
 // One 32-wide block: D = A_blk(16x32) * B(32x8) with A the exact integers,
 // two mma k-steps.  lo/hi: the lane's code words for this block.
-template <bool kBf16, int kBits>
+template <int kBits>
 __device__ __forceinline__ void block_mma(float (&d)[4], uint32_t lo, uint32_t hi, int hshift,
                                           uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
     uint32_t a[4];
     const float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int r = 0; r < 4; r++) a[r] = dq_pair<kBf16, kBits>(lo, hi, r, hshift);
-    if (kBf16) mma_bf16(d, a, b0, b1, z); else mma_f16(d, a, b0, b1, z);
+    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, r, hshift);
+    mma_f16(d, a, b0, b1, z);
 #pragma unroll
-    for (int r = 0; r < 4; r++) a[r] = dq_pair<kBf16, kBits>(lo, hi, 4 + r, hshift);
-    if (kBf16) mma_bf16(d, a, b2, b3, d); else mma_f16(d, a, b2, b3, d);
+    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, 4 + r, hshift);
+    mma_f16(d, a, b2, b3, d);
 }
 
 // Accumulate one 16 x (ns*128) slab of a matrix whose units sit in smem at
-// `w` against B rows staged at `xb` (row pitch `pitch` elements).
-template <bool kBf16, int kBits>
+// `w` against the fp16 token rows staged at `xb` (row pitch `pitch` elements,
+// `xrows` rows staged; the other mma columns read row 0 and are ignored).
+template <int kBits>
 __device__ __forceinline__ void slab_dot(float (&acc)[4], const uint8_t *w, int ns,
-                                         const uint16_t *xb, int pitch, int lane) {
+                                         const uint16_t *xb, int pitch, int xrows, int lane) {
     constexpr int UB = unit_bytes(kBits);
     constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
+    const uint16_t *xrow = xb + ((lane & 7) < xrows ? (lane & 7) : 0) * pitch;
     for (int sg = 0; sg < ns; sg++) {
         const uint8_t *un = w + sg * UB;
         uint4 lo = *reinterpret_cast<const uint4 *>(un + lane * 16);
@@ -60,11 +65,14 @@ __device__ __forceinline__ void slab_dot(float (&acc)[4], const uint8_t *w, int 
 #pragma unroll
         for (int blk = 0; blk < 4; blk++) {
             uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(b0, b1, b2, b3, xb + (lane & 7) * pitch + sg * 128 + blk * 32 + (lane >> 3) * 8);
+            ldmatrix_x4(b0, b1, b2, b3, xrow + sg * 128 + blk * 32 + (lane >> 3) * 8);
             uint32_t s2 = __shfl_sync(0xffffffffu, sc, (lane & ~3) | blk);
             float d[4];
-            block_mma<kBf16, kBits>(d, comp4(lo, blk), blk < 2 ? hi.x : hi.y, 8 * (blk & 1), b0, b1,
-                                    b2, b3);
+            if (kBits == 2)
+                block_mma2(d, comp4(lo, blk), b0, b1, b2, b3);
+            else
+                block_mma<kBits>(d, comp4(lo, blk), blk < 2 ? hi.x : hi.y, 8 * (blk & 1), b0, b1,
+                                 b2, b3);
             float2 s = __half22float2(*reinterpret_cast<__half2 *>(&s2));
             acc[0] = fmaf(s.x, d[0], acc[0]);
             acc[1] = fmaf(s.x, d[1], acc[1]);
@@ -79,15 +87,29 @@ template <int kBits>
 __global__ __launch_bounds__(128) void gemv_gateup_kernel(
     const uint8_t *__restrict__ routed, const uint8_t *__restrict__ shared, size_t expert_bytes,
     size_t mat_bytes, const int4 *__restrict__ units, const int *__restrict__ n_units,
-    const int32_t *__restrict__ list, int Tk, int E, const __nv_bfloat16 *__restrict__ x, int H,
-    int Ip, __half *__restrict__ a_out, int *err, long long budget) {
+    const int32_t *__restrict__ list, int Tk, int T, int E, const __nv_bfloat16 *__restrict__ x,
+    int H, int Ip, int xrows, int nsh, __half *__restrict__ a_out, int *err, long long budget) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ float red[4][32][8];
     constexpr int UB = unit_bytes(kBits);
     const int nslab = Ip / kSlabRows;
     const int u = blockIdx.x / nslab, slab = blockIdx.x % nslab;
-    if (u >= *n_units) return;
-    const int4 un = units[u];
+    // The first nsh units are the shared expert's, fixed before routing: those
+    // CTAs fetch weights and tokens while the routing kernel still runs.  The
+    // others wait for routing (programmatic dependent launch).
+    // Routed CTAs signal the down kernel only after their wait, i.e. once
+    // routing is complete, so the down kernel may read the unit list early;
+    // shared CTAs signal by exiting.
+    int4 un;
+    if (u < nsh) {
+        const int n0 = T - u * kTile;
+        un = make_int4(E, Tk + u * kTile, n0 < kTile ? n0 : kTile, 0);
+    } else {
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (u >= *n_units) return;
+        un = units[u];
+    }
     const int e = un.x, slot0 = un.y, n = un.z;
     const uint8_t *wg = e == E ? shared : routed + (size_t)e * expert_bytes;
     const uint8_t *wu = wg + mat_bytes;
@@ -98,7 +120,7 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
     const int wbytes = 2 * nsw * UB;
     const int pitch = nsw * kSegCols + 8;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    uint8_t *wbuf = smem + 128 + warp * (wbytes + kTile * pitch * 2);
+    uint8_t *wbuf = smem + 128 + warp * (wbytes + xrows * pitch * 2);
     uint16_t *xb = reinterpret_cast<uint16_t *>(wbuf + wbytes);
 
     if (lane == 0) {
@@ -114,23 +136,45 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
             mbar_arrive(&bars[warp]);
         }
     }
-    // stage the unit's token rows (this warp's column range), zero the rest
-    for (int j = 0; j < kTile; j++) {
-        uint4 *dst = reinterpret_cast<uint4 *>(xb + j * pitch);
-        if (j < n) {
-            int slot = slot0 + j;
-            int t = slot < Tk ? list[slot] : slot - Tk;
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H + sa * kSegCols);
-            for (int i = lane; i < ns * 16; i += 32) dst[i] = __ldg(src + i);
-        } else {
-            for (int i = lane; i < ns * 16; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+    // stage the unit's token rows (this warp's column range) as fp16, zero the
+    // rest; each lane requests a batch of 8 chunks before storing any
+    {
+        const int per_row = ns * 16, nchunk = xrows * per_row;
+        for (int base = 0; base < nchunk; base += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const int idx = base + b * 32 + lane;
+                v[b] = make_uint4(0, 0, 0, 0);
+                if (idx < nchunk) {
+                    const int j = idx / per_row, i = idx % per_row;
+                    if (j < n) {
+                        const int slot = slot0 + j;
+                        const int t = slot < Tk ? list[slot] : slot - Tk;
+                        v[b] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H +
+                                                                     sa * kSegCols) + i);
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const int idx = base + b * 32 + lane;
+                if (idx >= nchunk) break;
+                const int j = idx / per_row, i = idx % per_row;
+                const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&v[b]);
+                uint4 o;
+                __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+                for (int q = 0; q < 4; q++) h[q] = __float22half2_rn(__bfloat1622float2(bb[q]));
+                reinterpret_cast<uint4 *>(xb + j * pitch)[i] = o;
+            }
         }
     }
     __syncwarp();
     float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
     if (mbar_wait(&bars[warp], 0, budget, err)) {
-        slab_dot<true, kBits>(accg, wbuf, ns, xb, pitch, lane);
-        slab_dot<true, kBits>(accu, wbuf + nsw * UB, ns, xb, pitch, lane);
+        slab_dot<kBits>(accg, wbuf, ns, xb, pitch, xrows, lane);
+        slab_dot<kBits>(accu, wbuf + nsw * UB, ns, xb, pitch, xrows, lane);
     } else {
         mbar_drain(&bars[warp], 0);
     }
@@ -163,14 +207,18 @@ template <int kBits>
 __global__ __launch_bounds__(128) void gemv_down_kernel(
     const uint8_t *__restrict__ routed, const uint8_t *__restrict__ shared, size_t expert_bytes,
     size_t mat_bytes, const int4 *__restrict__ units, const int *__restrict__ n_units, int E,
-    const __half *__restrict__ a, int H, int Ip, float *__restrict__ Y, int *err,
+    const __half *__restrict__ a, int H, int Ip, int xrows, float *__restrict__ Y, int *err,
     long long budget) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int UB = unit_bytes(kBits);
     const int ngrp = H / 64;
     const int u = blockIdx.x / ngrp, grp = blockIdx.x % ngrp;
-    if (u >= *n_units) return;
-    const int4 un = units[u];
+    grid_launch_dependents();
+    // Routing finished before the gate/up kernel let this grid start, so the
+    // unit list is final; read it past L1 and fetch the weights before waiting
+    // for gate/up's activations.
+    if (u >= __ldcg(n_units)) return;
+    const int4 un = __ldcg(units + u);
     const int e = un.x, slot0 = un.y, n = un.z;
     const uint8_t *wd = (e == E ? shared : routed + (size_t)e * expert_bytes) + 2 * mat_bytes;
     const int nseg = Ip / kSegCols;
@@ -188,20 +236,31 @@ __global__ __launch_bounds__(128) void gemv_down_kernel(
         mbar_arrive_expect_tx(&bars[warp], bytes);
         bulk_g2s(wbuf, wd + (size_t)slab * nseg * UB, bytes, &bars[warp]);
     }
-    for (int j = 0; j < kTile; j++) {
-        uint4 *dst = reinterpret_cast<uint4 *>(ab + j * pitch);
-        const int nv = Ip / 8;
-        if (j < n) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a + (size_t)(slot0 + j) * Ip);
-            for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = src[i];
-        } else {
-            for (int i = threadIdx.x; i < nv; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    grid_dependency_wait();  // gate/up's activations
+    {
+        const int nv = Ip / 8, nchunk = xrows * nv;
+        for (int base = 0; base < nchunk; base += 8 * 128) {
+            uint4 v[8];
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const int idx = base + b * 128 + threadIdx.x;
+                v[b] = make_uint4(0, 0, 0, 0);
+                if (idx < nchunk && idx / nv < n)
+                    v[b] = __ldcg(reinterpret_cast<const uint4 *>(a + (size_t)(slot0 + idx / nv) * Ip) +
+                                  idx % nv);
+            }
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const int idx = base + b * 128 + threadIdx.x;
+                if (idx >= nchunk) break;
+                reinterpret_cast<uint4 *>(ab + (idx / nv) * pitch)[idx % nv] = v[b];
+            }
         }
     }
     __syncthreads();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (mbar_wait(&bars[warp], 0, budget, err)) {
-        slab_dot<false, kBits>(acc, wbuf, nseg, ab, pitch, lane);
+        slab_dot<kBits>(acc, wbuf, nseg, ab, pitch, xrows, lane);
     } else {
         mbar_drain(&bars[warp], 0);
     }
@@ -214,48 +273,41 @@ __global__ __launch_bounds__(128) void gemv_down_kernel(
     }
 }
 
-static size_t gateup_smem(const Geometry &g) {
+static int staged_rows(int T) { return T < kTile ? (T < 1 ? 1 : T) : kTile; }
+
+static size_t gateup_smem(const Geometry &g, int xrows) {
     int nseg = g.H / kSegCols, nsw = (nseg + 3) / 4;
-    return 128 + 4 * (size_t)(2 * nsw * g.ub + kTile * (nsw * kSegCols + 8) * 2);
+    return 128 + 4 * (size_t)(2 * nsw * g.ub + xrows * (nsw * kSegCols + 8) * 2);
 }
 
-static size_t down_smem(const Geometry &g) {
-    return 128 + 4 * (size_t)g.nseg_i * g.ub + (size_t)kTile * (g.Ip + 8) * 2;
+static size_t down_smem(const Geometry &g, int xrows) {
+    return 128 + 4 * (size_t)g.nseg_i * g.ub + (size_t)xrows * (g.Ip + 8) * 2;
 }
 
 void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                        const int *n_units, int units_max, const int32_t *list, int Tk,
+                        const int *n_units, int units_max, const int32_t *list, int Tk, int T,
                         const void *x, void *a_out, int *err, long long budget, cudaStream_t s) {
-    size_t smem = gateup_smem(g);
+    const int xrows = staged_rows(T);
+    const int nsh = (T + kTile - 1) / kTile;
+    size_t smem = gateup_smem(g, xrows);
     dim3 grid((unsigned)((size_t)units_max * (g.Ip / kSlabRows)));
     auto xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     auto ao = reinterpret_cast<__half *>(a_out);
-    if (g.bits == 2) {
-        gemv_gateup_kernel<2><<<grid, 128, smem, s>>>(w.routed, w.shared, g.expert_bytes,
-                                                      g.mat_bytes, units, n_units, list, Tk, g.E,
-                                                      xb, g.H, g.Ip, ao, err, budget);
-    } else {
-        gemv_gateup_kernel<3><<<grid, 128, smem, s>>>(w.routed, w.shared, g.expert_bytes,
-                                                      g.mat_bytes, units, n_units, list, Tk, g.E,
-                                                      xb, g.H, g.Ip, ao, err, budget);
-    }
+    auto kern = g.bits == 2 ? gemv_gateup_kernel<2> : gemv_gateup_kernel<3>;
+    launch_pdl(kern, grid, dim3(128), smem, s, w.routed, w.shared, g.expert_bytes, g.mat_bytes,
+               units, n_units, list, Tk, T, g.E, xb, g.H, g.Ip, xrows, nsh, ao, err, budget);
 }
 
 void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                      const int *n_units, int units_max, const void *a, float *Y, int *err,
+                      const int *n_units, int units_max, int T, const void *a, float *Y, int *err,
                       long long budget, cudaStream_t s) {
-    size_t smem = down_smem(g);
+    const int xrows = staged_rows(T);
+    size_t smem = down_smem(g, xrows);
     dim3 grid((unsigned)((size_t)units_max * (g.H / 64)));
     auto ap = reinterpret_cast<const __half *>(a);
-    if (g.bits == 2) {
-        gemv_down_kernel<2><<<grid, 128, smem, s>>>(w.routed, w.shared, g.expert_bytes,
-                                                    g.mat_bytes, units, n_units, g.E, ap, g.H,
-                                                    g.Ip, Y, err, budget);
-    } else {
-        gemv_down_kernel<3><<<grid, 128, smem, s>>>(w.routed, w.shared, g.expert_bytes,
-                                                    g.mat_bytes, units, n_units, g.E, ap, g.H,
-                                                    g.Ip, Y, err, budget);
-    }
+    auto kern = g.bits == 2 ? gemv_down_kernel<2> : gemv_down_kernel<3>;
+    launch_pdl(kern, grid, dim3(128), smem, s, w.routed, w.shared, g.expert_bytes, g.mat_bytes,
+               units, n_units, g.E, ap, g.H, g.Ip, xrows, Y, err, budget);
 }
 
 cudaError_t gemv_init_attributes(int max_smem) {

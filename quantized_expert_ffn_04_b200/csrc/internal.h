@@ -1,6 +1,7 @@
 // Host-side declarations shared by the library's .cu files (not part of the ABI).
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -50,26 +51,46 @@ void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int3
                      int32_t *list, int32_t *slot, const DispatchScratch &ds, int4 *units,
                      int *n_units, int tile, cudaStream_t s);
 
+// Top-k + dispatch for T <= kSmallMaxT tokens in a single CTA.
+constexpr int kSmallMaxT = 256;
+void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                        int32_t *cnt, int32_t *off, int32_t *list, int32_t *slot, int4 *units,
+                        int *n_units, int tile, cudaStream_t s);
+
+// Large batches: screened top-k from the split-weight screening GEMM D
+// ([T][R], hi part in columns [0, E), lo part in [E, 2E)) and exact recompute
+// of the candidates (see route.cu for the bound).
+void launch_screen_topk(const float *D, int R, const void *x, int T, int H, const float *Wp,
+                        const float *bias, int E, int k, float gam, float wmax, float bmax,
+                        int32_t *idx, float *w, cudaStream_t s);
+
 // ---- gemv.cu (decode)
 struct ExpertWeights {
     const uint8_t *routed;   // expert e at routed + e * expert_bytes
     const uint8_t *shared;   // the shared expert
 };
 void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                        const int *n_units, int units_max, const int32_t *list, int Tk,
+                        const int *n_units, int units_max, const int32_t *list, int Tk, int T,
                         const void *x, void *a_out, int *err, long long budget, cudaStream_t s);
 void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                      const int *n_units, int units_max, const void *a, float *Y, int *err,
+                      const int *n_units, int units_max, int T, const void *a, float *Y, int *err,
                       long long budget, cudaStream_t s);
 
 // ---- umma.cu (prefill)
 // x (bf16) -> x16 (fp16 copy), then gate/up (a: fp16 [slots][Ip]) and down
 // (Y: fp16 [slots][H]) on the tensor cores.  Units of up to 256 tokens.
 constexpr int kUmmaTile = 256;
-void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                         const int *n_units, int units_max, const int32_t *list, int Tk,
-                         const void *x, void *x16, void *a, void *Y, int *err, long long budget,
-                         int T, cudaStream_t s);
+void launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                        const int *n_units, int units_max, const int32_t *list, int Tk,
+                        const void *x16, void *a, int *err, long long budget, cudaStream_t s);
+void launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                      const int *n_units, int units_max, const void *a, void *Y, int *err,
+                      long long budget, cudaStream_t s);
+// Plain fp16 GEMM on the tensor cores: D[t][r] = sum_k x16[t][k] * A[r][k],
+// rows a multiple of 128, K a multiple of 128; fp32 out with row stride `rows`.
+void launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
+                       int *err, long long budget, cudaStream_t s);
+void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s);
 cudaError_t umma_init_attributes(int max_smem);
 
 // ---- combine.cu
@@ -83,6 +104,25 @@ void launch_rmsnorm(const void *h, void *xn, int T, int H, cudaStream_t s);
 
 // ---- selftest
 void launch_selftest_wait(int *err, long long budget, cudaStream_t s);
+
+// Launch `kernel` so that it may begin while the previous kernel of the stream
+// drains (programmatic dependent launch); the kernel calls
+// grid_dependency_wait() before it reads anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // Set the thread-local message returned by strata_moe_last_error().
 void set_error_message(const char *msg);

@@ -45,7 +45,7 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes,
             for (int half = 0; half < 2; half++) {
                 int col = col0 + half;
                 int q = (row < R && col < K) ? canon_code(codes, bits, K, row, col) : 0;
-                lo[w] |= (uint32_t)(q & 3) << (2 * rp + 16 * half);
+                lo[w] |= (uint32_t)(q & 3) << (code_pos(bits, rp) + 16 * half);
                 if (bits == 3)
                     hi[w >> 1] |= (uint32_t)((q >> 2) & 1) << (rp + 8 * (w & 1) + 16 * half);
             }
@@ -101,12 +101,14 @@ __device__ float debug_weight(const uint8_t *mat, int Kp, int row, int col, int 
     uint16_t dbits = (uint16_t)(rr >= 8 ? (sw >> 16) : (sw & 0xffff));
     __half d = __ushort_as_half(dbits);
     if (kind == 0) {
-        uint32_t p = dq_pair<true, kBits>(lo, hi, rp, 8 * (w & 1));
-        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&p);
-        float q2 = half ? __high2float(v) : __low2float(v);  // 2q - (2^bits - 1), exact
-        return q2 * (__half2float(d) * 0.5f);                 // exact in fp32
+        // the code read straight from its bit position, then 2q - (2^bits - 1)
+        int q = (lo >> (code_pos(kBits, rp) + 16 * half)) & 3;
+        if (kBits == 3) q |= ((hi >> (rp + 8 * (w & 1) + 16 * half)) & 1) << 2;
+        const float q2 = (float)(2 * q - ((1 << kBits) - 1));
+        return q2 * (__half2float(d) * 0.5f);  // exact in fp32
     } else {
-        uint32_t p = dq_pair<false, kBits>(lo, hi, rp, 8 * (w & 1));
+        // the tensor-core operand, computed by the prefill kernels' routine
+        uint32_t p = kBits == 2 ? dq2_pair(lo, rp) : dq_pair<false, kBits>(lo, hi, rp, 8 * (w & 1));
         __half2 v = *reinterpret_cast<__half2 *>(&p);
         __half dh = __hmul(d, __float2half(0.5f));
         __half2 wv = __hmul2(v, __half2half2(dh));

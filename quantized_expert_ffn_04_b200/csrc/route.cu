@@ -26,7 +26,7 @@ namespace strata {
 // fixed order; TT tokens per CTA staged in smem as fp32 in the same
 // lane-interleaved layout as the weights: xs[tt][s4][lane] = float4 of
 // x[128*s4 + 32*j + lane], j = 0..3.
-template <int TT, int EE>
+template <int TT, int EE, int CH>
 __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__restrict__ x, int T,
                                                      int H, const float4 *__restrict__ Wp,
                                                      const float *__restrict__ bias, int E,
@@ -34,19 +34,33 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
     extern __shared__ float4 xs[];
     const int ns4 = H / 128;
     const int t0 = blockIdx.y * TT;
-    // stage TT token rows (16 bytes = 8 bf16 per step)
-    for (int idx = threadIdx.x; idx < TT * H / 8; idx += blockDim.x) {
-        int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
-        int t = t0 + tt;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < T) v = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + i0);
-        const __nv_bfloat16 *pv = reinterpret_cast<const __nv_bfloat16 *>(&v);
-        float *xf = reinterpret_cast<float *>(xs);
+    // stage TT token rows (16 bytes = 8 bf16 per chunk); each thread requests a
+    // batch of 8 chunks before storing any, so the loads overlap
+    const int nchunk = TT * H / 8;
+    float *xf = reinterpret_cast<float *>(xs);
+    for (int base = 0; base < nchunk; base += 8 * blockDim.x) {
+        uint4 v[8];
 #pragma unroll
-        for (int q = 0; q < 8; q++) {
-            int i = i0 + q;
-            xf[(((size_t)tt * ns4 + (i >> 7)) * 32 + (i & 31)) * 4 + ((i >> 5) & 3)] =
-                __bfloat162float(pv[q]);
+        for (int b = 0; b < 8; b++) {
+            const int idx = base + b * blockDim.x + threadIdx.x;
+            v[b] = make_uint4(0, 0, 0, 0);
+            if (idx < nchunk) {
+                const int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
+                if (t0 + tt < T) v[b] = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H + i0);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < 8; b++) {
+            const int idx = base + b * blockDim.x + threadIdx.x;
+            if (idx >= nchunk) break;
+            const int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
+            const __nv_bfloat16 *pv = reinterpret_cast<const __nv_bfloat16 *>(&v[b]);
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int i = i0 + q;
+                xf[(((size_t)tt * ns4 + (i >> 7)) * 32 + (i & 31)) * 4 + ((i >> 5) & 3)] =
+                    __bfloat162float(pv[q]);
+            }
         }
     }
     __syncthreads();
@@ -59,24 +73,32 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
 #pragma unroll
         for (int b = 0; b < EE; b++) acc[a][b] = 0.0f;
 
-#pragma unroll 2
-    for (int s4 = 0; s4 < ns4; s4++) {
-        float4 wv[EE];
+    // CH steps of weights are requested before any of them is used, so a warp
+    // keeps CH x EE x 512 bytes in flight.
+    for (int s0 = 0; s0 < ns4; s0 += CH) {
+        float4 wv[CH][EE];
 #pragma unroll
-        for (int b = 0; b < EE; b++) {
-            int e = e0 + b;
-            wv[b] = e < E ? __ldg(Wp + ((size_t)e * ns4 + s4) * 32 + lane)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int a = 0; a < TT; a++) {
-            float4 xv = xs[((size_t)a * ns4 + s4) * 32 + lane];
+        for (int c = 0; c < CH; c++)
 #pragma unroll
             for (int b = 0; b < EE; b++) {
-                acc[a][b] = fmaf(xv.x, wv[b].x, acc[a][b]);
-                acc[a][b] = fmaf(xv.y, wv[b].y, acc[a][b]);
-                acc[a][b] = fmaf(xv.z, wv[b].z, acc[a][b]);
-                acc[a][b] = fmaf(xv.w, wv[b].w, acc[a][b]);
+                int e = e0 + b, s4 = s0 + c;
+                wv[c][b] = (e < E && s4 < ns4) ? __ldg(Wp + ((size_t)e * ns4 + s4) * 32 + lane)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+        for (int c = 0; c < CH; c++) {
+            const int s4 = s0 + c;
+            if (s4 >= ns4) break;
+#pragma unroll
+            for (int a = 0; a < TT; a++) {
+                float4 xv = xs[((size_t)a * ns4 + s4) * 32 + lane];
+#pragma unroll
+                for (int b = 0; b < EE; b++) {
+                    acc[a][b] = fmaf(xv.x, wv[c][b].x, acc[a][b]);
+                    acc[a][b] = fmaf(xv.y, wv[c][b].y, acc[a][b]);
+                    acc[a][b] = fmaf(xv.z, wv[c][b].z, acc[a][b]);
+                    acc[a][b] = fmaf(xv.w, wv[c][b].w, acc[a][b]);
+                }
             }
         }
     }
@@ -104,11 +126,11 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
     }
 }
 
-template <int TT, int EE>
+template <int TT, int EE, int CH>
 static void run_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
                        float *logits, cudaStream_t s) {
     size_t smem = (size_t)TT * H * sizeof(float);
-    auto kern = router_kernel<TT, EE>;
+    auto kern = router_kernel<TT, EE, CH>;
     dim3 grid((E + 4 * EE - 1) / (4 * EE), (T + TT - 1) / TT);
     kern<<<grid, 128, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
                                  reinterpret_cast<const float4 *>(Wp), bias, E, logits);
@@ -117,13 +139,13 @@ static void run_router(const void *x, int T, int H, const float *Wp, const float
 void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
                    float *logits, cudaStream_t s) {
     if (T <= 1)
-        run_router<1, 1>(x, T, H, Wp, bias, E, logits, s);
+        run_router<1, 1, 20>(x, T, H, Wp, bias, E, logits, s);
     else if (T <= 4)
-        run_router<4, 1>(x, T, H, Wp, bias, E, logits, s);
+        run_router<4, 1, 20>(x, T, H, Wp, bias, E, logits, s);
     else if (T <= 64)
-        run_router<8, 2>(x, T, H, Wp, bias, E, logits, s);
+        run_router<8, 2, 8>(x, T, H, Wp, bias, E, logits, s);
     else
-        run_router<8, 8>(x, T, H, Wp, bias, E, logits, s);
+        run_router<8, 8, 2>(x, T, H, Wp, bias, E, logits, s);
 }
 
 // ============================================================== top-k
@@ -133,13 +155,11 @@ __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
     return va > vb || (va == vb && ea < eb);
 }
 
-__global__ __launch_bounds__(256) void topk_kernel(const float *__restrict__ logits, int T, int E,
-                                                   int k, int32_t *__restrict__ idx,
-                                                   float *__restrict__ wout) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
-    if (t >= T) return;
-    const float *row = logits + (size_t)t * E;
+// Top-k of one token's logits by one warp; lane j < k ends with pick j.
+// Writes idx/w (global) and, when sidx != nullptr, the picks to shared memory.
+__device__ __forceinline__ void topk_token(const float *__restrict__ row, int E, int k, int lane,
+                                           int32_t *__restrict__ idx, float *__restrict__ wout,
+                                           int *sidx) {
     const int nq = (E + 31) >> 5;  // <= 32
     float v[32];
 #pragma unroll
@@ -183,9 +203,20 @@ __global__ __launch_bounds__(256) void topk_kernel(const float *__restrict__ log
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane < k) {
-        idx[(size_t)t * k + lane] = my_e;
-        wout[(size_t)t * k + lane] = ex / sum;
+        idx[lane] = my_e;
+        wout[lane] = ex / sum;
+        if (sidx) sidx[lane] = my_e;
     }
+}
+
+__global__ __launch_bounds__(256) void topk_kernel(const float *__restrict__ logits, int T, int E,
+                                                   int k, int32_t *__restrict__ idx,
+                                                   float *__restrict__ wout) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= T) return;
+    topk_token(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, wout + (size_t)t * k,
+               nullptr);
 }
 
 void launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
@@ -319,15 +350,17 @@ __global__ __launch_bounds__(1024) void dispatch_scan_kernel(int T, int k, int E
     int nu = e < E ? (ce + tile - 1) / tile : 0;
     int utot;
     int us = block_exclusive_scan(nu, &utot);
+    // shared-expert units first (their position is known before routing), then
+    // the routed experts' units in ascending expert id
+    int nsh = (T + tile - 1) / tile;
     if (e < E)
         for (int i = 0; i < nu; i++) {
             int n = ce - i * tile;
-            units[us + i] = make_int4(e, oe + i * tile, n < tile ? n : tile, 0);
+            units[nsh + us + i] = make_int4(e, oe + i * tile, n < tile ? n : tile, 0);
         }
-    int nsh = (T + tile - 1) / tile;
     for (int i = threadIdx.x; i < nsh; i += blockDim.x) {
         int n = T - i * tile;
-        units[utot + i] = make_int4(E, T * k + i * tile, n < tile ? n : tile, 0);
+        units[i] = make_int4(E, T * k + i * tile, n < tile ? n : tile, 0);
     }
     if (threadIdx.x == 0) *n_units = utot + nsh;
 }
@@ -363,12 +396,283 @@ void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int3
     dispatch_scatter_kernel<<<nc, 256, 0, s>>>(idx, T, k, E, ds.hist, ds.bm, ds.pre, list, slot);
 }
 
+// ============================================================== screened top-k
+// Large batches: the router's tensor-core screening GEMM gives approximate
+// logits a_e = x . (W_hi + W_lo)_e (+ b_e), with W_hi = fp16(W) and
+// W_lo = fp16(W - W_hi).  With the bound |a_e - l_e| <= eps for the exact
+// fixed-order logits l_e, every expert of the exact top-k has
+// a_e >= a_(k) - 2 eps (a_(k): k-th largest approximate logit; a tie at the
+// boundary is included too).  Those candidates are recomputed exactly in the
+// fixed order and the top-k is taken among them, so the picks and weights are
+// the same bits as with the full fp32 router.
+//
+// eps (per token) = 2 x [ (H 2^-23 + 2^-22 + (H/32 + 10) 2^-24) ||x||_2 max_e ||W_e||_2
+//                         + 2^-25 ||x||_1 + 2^-22 max_e |b_e| ]:
+// tensor-core fp32 accumulation of H exact products (truncating adder assumed),
+// the two-term fp16 split (relative 2^-22 plus a subnormal quantum 2^-25), the
+// fixed-order fp32 sum and the bias additions, with |x|.|W_e| <= ||x|| ||W_e||;
+// the leading 2 is a safety factor.  The screening GEMM reads the fp16 copy of
+// x: bf16 -> fp16 is exact for 2^-14 <= |x| <= 65504 and off by at most 2^-25
+// below, adding 2^-25 ||W_e||_1 <= 2^-25 sqrt(H) ||W_e||_2; a token with any
+// |x| > 65504 (or a non-finite bound) keeps every expert as a candidate.
+
+// k picks among the lanes' values v (lane l holds experts l, l+32, ...);
+// experts whose bit is set in `taken` are excluded.  Lane j < k ends with pick
+// j; writes idx/w.
+__device__ __forceinline__ void select_topk(const float (&v)[32], uint32_t taken, int E, int k,
+                                            int lane, int32_t *__restrict__ idx,
+                                            float *__restrict__ wout) {
+    const int nq = (E + 31) >> 5;
+    float my_v = -INFINITY;
+    int my_e = -1;
+    for (int j = 0; j < k; j++) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 32; q++) {
+            int e = q * 32 + lane;
+            if (q < nq && e < E && !((taken >> q) & 1) && better(v[q], e, bv, be)) {
+                bv = v[q];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (better(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) {
+            my_v = bv;
+            my_e = be;
+        }
+    }
+    float m = __shfl_sync(0xffffffffu, my_v, 0);
+    float ex = lane < k ? expf(my_v - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+        idx[lane] = my_e;
+        wout[lane] = ex / sum;
+    }
+}
+
+__global__ __launch_bounds__(128) void screen_topk_kernel(
+    const float *__restrict__ D, int R, const __nv_bfloat16 *__restrict__ x, int T, int H,
+    const float4 *__restrict__ Wp, const float *__restrict__ bias, int E, int k, float gam,
+    float wmax, float bmax, int32_t *__restrict__ idx, float *__restrict__ wout) {
+    extern __shared__ float4 sm4[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 4 + warp;
+    if (t >= T) return;
+    const int ns4 = H / 128;
+    float4 *xs = sm4 + (size_t)warp * (H / 4);
+    float *exl = reinterpret_cast<float *>(sm4 + 4 * (H / 4)) + warp * 1024;
+    // token row in the router's lane-interleaved fp32 layout, and its norms
+    float ss = 0.f, s1 = 0.f, xm = 0.f;
+    const __nv_bfloat16 *xr = x + (size_t)t * H;
+    for (int s4 = 0; s4 < ns4; s4++) {
+        float v0 = __bfloat162float(xr[128 * s4 + lane]);
+        float v1 = __bfloat162float(xr[128 * s4 + 32 + lane]);
+        float v2 = __bfloat162float(xr[128 * s4 + 64 + lane]);
+        float v3 = __bfloat162float(xr[128 * s4 + 96 + lane]);
+        ss = fmaf(v0, v0, fmaf(v1, v1, fmaf(v2, v2, fmaf(v3, v3, ss))));
+        s1 += fabsf(v0) + fabsf(v1) + fabsf(v2) + fabsf(v3);
+        xm = fmaxf(xm, fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+        xs[s4 * 32 + lane] = make_float4(v0, v1, v2, v3);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, o));
+    }
+    __syncwarp();
+    const float eps =
+        2.0f * (gam * sqrtf(ss) * 1.001f * wmax + 2.9802322e-8f * s1 * 1.001f +
+                2.9802322e-8f * sqrtf((float)H) * wmax + 2.3841858e-7f * bmax);
+    const bool finite = isfinite(eps) && !(xm > 65504.0f);
+    const int nq = (E + 31) >> 5;
+    const float *dr = D + (size_t)t * R;
+    float av[32];
+#pragma unroll
+    for (int q = 0; q < 32; q++) {
+        int e = q * 32 + lane;
+        float a = -INFINITY;
+        if (q < nq && e < E) {
+            a = (dr[e] + dr[E + e]) + (bias ? bias[e] : 0.0f);
+            if (a != a) a = INFINITY;  // keep a NaN screening value as a candidate
+        }
+        av[q] = a;
+    }
+    // k-th largest approximate logit
+    uint32_t taken = 0;
+    float kth = INFINITY;
+    for (int j = 0; j < k; j++) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 32; q++) {
+            int e = q * 32 + lane;
+            if (q < nq && e < E && !((taken >> q) & 1) && better(av[q], e, bv, be)) {
+                bv = av[q];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (better(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        kth = bv;
+    }
+    const float thr = finite ? kth - 2.0f * eps : -INFINITY;
+    uint32_t cand = 0;
+#pragma unroll
+    for (int q = 0; q < 32; q++) {
+        int e = q * 32 + lane;
+        if (q < nq && e < E && (!(av[q] < thr))) cand |= 1u << q;
+    }
+    const uint32_t cset = cand;
+    // exact fixed-order logits of the candidates, one warp-wide dot product each
+    for (;;) {
+        const uint32_t any = __ballot_sync(0xffffffffu, cand != 0);
+        if (!any) break;
+        const int src = __ffs(any) - 1;
+        const int q = __shfl_sync(0xffffffffu, __ffs(cand) - 1, src);
+        if (lane == src) cand &= ~(1u << q);
+        const int e = 32 * q + src;
+        float pacc = 0.0f;
+        const float4 *wr = Wp + (size_t)e * ns4 * 32 + lane;
+        for (int s4 = 0; s4 < ns4; s4++) {
+            const float4 w = __ldg(wr + s4 * 32);
+            const float4 xv = xs[s4 * 32 + lane];
+            pacc = fmaf(xv.x, w.x, pacc);
+            pacc = fmaf(xv.y, w.y, pacc);
+            pacc = fmaf(xv.z, w.z, pacc);
+            pacc = fmaf(xv.w, w.w, pacc);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) pacc = __fadd_rn(pacc, __shfl_down_sync(0xffffffffu, pacc, o));
+        if (lane == 0) exl[e] = bias ? __fadd_rn(pacc, bias[e]) : pacc;
+    }
+    __syncwarp();
+    float v[32];
+#pragma unroll
+    for (int q = 0; q < 32; q++) {
+        int e = q * 32 + lane;
+        float lv = ((cset >> q) & 1) ? exl[e] : -INFINITY;
+        v[q] = lv != lv ? -INFINITY : lv;
+    }
+    select_topk(v, ~cset, E, k, lane, idx + (size_t)t * k, wout + (size_t)t * k);
+}
+
+void launch_screen_topk(const float *D, int R, const void *x, int T, int H, const float *Wp,
+                        const float *bias, int E, int k, float gam, float wmax, float bmax,
+                        int32_t *idx, float *w, cudaStream_t s) {
+    size_t smem = (size_t)4 * H * 4 + (size_t)4 * 1024 * 4;
+    screen_topk_kernel<<<(T + 3) / 4, 128, smem, s>>>(
+        D, R, reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
+        reinterpret_cast<const float4 *>(Wp), bias, E, k, gam, wmax, bmax, idx, w);
+}
+
+// ============================================================== small batches
+// Top-k and dispatch of up to 256 tokens in one CTA of 1024 threads: warps
+// take tokens w, w+32, ...; then the same bitmap ranking as the chunked
+// kernels, all in shared memory, with one launch instead of four.
+__global__ __launch_bounds__(1024) void route_small_kernel(
+    const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx,
+    float *__restrict__ wout, int32_t *__restrict__ cnt, int32_t *__restrict__ off,
+    int32_t *__restrict__ list, int32_t *__restrict__ slot, int4 *__restrict__ units,
+    int *__restrict__ n_units, int tile) {
+    extern __shared__ uint32_t sm[];
+    grid_launch_dependents();  // the shared expert's gate/up CTAs may start now
+    grid_dependency_wait();
+    uint32_t *bm = sm;                                      // [8][E]
+    int *pre = reinterpret_cast<int *>(bm + 8 * E);         // [8][E]
+    int *soff = pre + 8 * E;                                // [E]
+    int *sidx = soff + E;                                   // [T][k]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) bm[i] = 0;
+    for (int t = warp; t < T; t += 32)
+        topk_token(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, wout + (size_t)t * k,
+                   sidx + t * k);
+    __syncthreads();
+    if ((int)threadIdx.x < T) {
+        const int t = threadIdx.x;
+        for (int j = 0; j < k; j++) atomicOr(&bm[(t >> 5) * E + sidx[t * k + j]], 1u << (t & 31));
+    }
+    __syncthreads();
+    const int ng = (T + 31) >> 5;
+    const int e = threadIdx.x;  // E <= 1024
+    int ce = 0;
+    if (e < E)
+        for (int g = 0; g < ng; g++) {
+            pre[g * E + e] = ce;
+            ce += __popc(bm[g * E + e]);
+        }
+    int total;
+    const int oe = block_exclusive_scan(e < E ? ce : 0, &total);
+    if (e < E) {
+        cnt[e] = ce;
+        off[e] = oe;
+        soff[e] = oe;
+    }
+    if (e == 0) off[E] = total;
+    const int nu = e < E ? (ce + tile - 1) / tile : 0;
+    int utot;
+    const int us = block_exclusive_scan(nu, &utot);
+    // shared-expert units first, then routed experts in ascending id
+    const int nsh = (T + tile - 1) / tile;
+    if (e < E)
+        for (int i = 0; i < nu; i++) {
+            int n = ce - i * tile;
+            units[nsh + us + i] = make_int4(e, oe + i * tile, n < tile ? n : tile, 0);
+        }
+    for (int i = threadIdx.x; i < nsh; i += blockDim.x) {
+        int n = T - i * tile;
+        units[i] = make_int4(E, T * k + i * tile, n < tile ? n : tile, 0);
+    }
+    if (threadIdx.x == 0) *n_units = utot + nsh;
+    __syncthreads();
+    if ((int)threadIdx.x < T) {
+        const int t = threadIdx.x, g = t >> 5;
+        const uint32_t below = (1u << (t & 31)) - 1u;
+        for (int j = 0; j < k; j++) {
+            const int ej = sidx[t * k + j];
+            const int pos = soff[ej] + pre[g * E + ej] + __popc(bm[g * E + ej] & below);
+            list[pos] = t;
+            slot[(size_t)t * k + j] = pos;
+        }
+    }
+}
+
+void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                        int32_t *cnt, int32_t *off, int32_t *list, int32_t *slot, int4 *units,
+                        int *n_units, int tile, cudaStream_t s) {
+    size_t smem = ((size_t)8 * E * 2 + E + (size_t)T * k) * 4;
+    launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, s, logits, T, E, k, idx, w, cnt,
+               off, list, slot, units, n_units, tile);
+}
+
 cudaError_t route_init_attributes(int max_smem) {
     cudaError_t e;
-    if ((e = allow_max_dyn_smem(router_kernel<1, 1>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<4, 1>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<8, 2>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<8, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<1, 1, 20>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<4, 1, 20>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<8, 2, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<8, 8, 2>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(route_small_kernel, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(screen_topk_kernel, max_smem)) != cudaSuccess) return e;
     return allow_max_dyn_smem(dispatch_count_kernel, max_smem);
 }
 

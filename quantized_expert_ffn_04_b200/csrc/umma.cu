@@ -37,12 +37,17 @@ constexpr int kTileB = kTN * kKS * 2;   // 32 KB
 constexpr int kWarpMma = 0, kWarpLoadB = 1, kWarpDq0 = 2, kNumDq = 4, kNumEpi = 4;  // epilogue: warps 6..9
 constexpr int kUmmaThreads = 32 * 10;
 
-template <bool kGateUp>
+// Modes: gate/up (A = dequantised Wg and Wu, SwiGLU epilogue, fp16 out),
+// down (A = dequantised Wd, fp16 out), plain (A = an fp16 matrix copied with
+// cp.async, fp32 out; used by the router's screening GEMM).
+constexpr int kModeGateUp = 0, kModeDown = 1, kModePlain = 2;
+
+template <int kMode>
 struct UmmaCfg {
-    static constexpr int kMats = kGateUp ? 2 : 1;
-    static constexpr int kStages = kGateUp ? 3 : 4;
+    static constexpr int kMats = kMode == kModeGateUp ? 2 : 1;
+    static constexpr int kStages = kMode == kModeGateUp ? 3 : 4;
     static constexpr int kStageBytes = kMats * kTileA + kTileB;
-    static constexpr int kTmemCols = kGateUp ? 512 : 256;
+    static constexpr int kTmemCols = kMode == kModeGateUp ? 512 : 256;
     static constexpr int kSmem = kStages * kStageBytes + 2048;
 };
 
@@ -55,13 +60,24 @@ struct UmmaParams {
     int E;
     const int32_t *list;
     int Tk;
-    const __half *xin;  // gate/up: x as fp16 [T][K]; down: a [slots][K]
+    const __half *xin;  // gate/up: x as fp16 [T][K]; down: a [slots][K]; plain: x [T][K]
     int K, nseg, n_rt;
     __half *out;        // gate/up: a [slots][Ip]; down: Y [slots][H]
+    float *out32;       // plain: D [T][n_rt * 128]
+    const __half *aplain;  // plain: A [n_rt * 128][K] fp16
+    int direct_T;       // plain: tiles are tokens [256u, 256u + 256) of T tokens
     int out_ld;
     int *err;
     long long budget;
 };
+
+__device__ __forceinline__ int4 tile_unit(const UmmaParams &p, int u) {
+    if (p.direct_T > 0) {
+        const int s0 = u * kTN, n = p.direct_T - s0;
+        return make_int4(0, s0, n < kTN ? n : kTN, 0);
+    }
+    return p.units[u];
+}
 
 __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long long budget,
                                           int *err, volatile int *abort_flag) {
@@ -71,7 +87,7 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long l
         return false;
     }
     long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > budget) {
             atomicCAS(err, 0, kErrTimeout);
@@ -85,9 +101,10 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long l
 __device__ __forceinline__ uint32_t h2u(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
 __device__ __forceinline__ __half2 u2h(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
 
-template <int kBits, bool kGateUp>
+template <int kBits, int kMode>
 __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const UmmaParams p) {
-    using Cfg = UmmaCfg<kGateUp>;
+    constexpr bool kGateUp = kMode == kModeGateUp;
+    using Cfg = UmmaCfg<kMode>;
     constexpr int S = Cfg::kStages, SB = Cfg::kStageBytes;
     constexpr int UB = unit_bytes(kBits);
     constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
@@ -124,7 +141,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_tiles = *p.n_units * p.n_rt;
+    const int n_tiles =
+        (p.direct_T > 0 ? (p.direct_T + kTN - 1) / kTN : *p.n_units) * p.n_rt;
     const int ksteps = p.K / kKS;
 
     if (warp == kWarpMma) {
@@ -134,7 +152,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, it++) {
-                const int n = p.units[t / p.n_rt].z;
+                const int n = tile_unit(p, t / p.n_rt).z;
                 const uint32_t idesc = umma_idesc_f16(kTM, (n + 15) & ~15);
                 if (it > 0 && !pipe_wait(acc_empty, (it - 1) & 1, p.budget, p.err, abort_flag)) break;
                 tc_fence_after();
@@ -172,7 +190,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
         int prev = -1;
         const int crow = lane >> 3, chunk = lane & 7;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-            const int4 un = p.units[t / p.n_rt];
+            const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
             const int rows = (n + 15) & ~15;
             // the previous tile's stages only read rowoff while issuing, so it
@@ -221,19 +239,17 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
             __syncwarp();
             if (lane == 0) mbar_arrive(&full_b[prev]);
         }
-    } else if (warp < kWarpDq0 + kNumDq) {
-        // ---------------------------------------------------------- dequant
-        const int dt = threadIdx.x - 32 * kWarpDq0;  // 0..127
-        const int L = dt & 31, sl0 = dt >> 5;        // slabs sl0 and sl0 + 4
-        const int g8 = L >> 2, c = L & 3;
-        const __half2 half2_05 = __float2half2_rn(0.5f);
+    } else if (kMode == kModePlain && warp < kWarpDq0 + kNumDq) {
+        // ---------------------------------------------------------- A copy
+        // 128 rows x 64 columns of fp16 per stage: 1024 16-byte chunks, each one
+        // row of one core matrix; 8 per thread, grouped per stage.
+        const int dt = threadIdx.x - 32 * kWarpDq0;
         uint32_t gs = 0;
+        int prev = -1;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const int rt = t % p.n_rt;
-            const int e = p.units[t / p.n_rt].x;
-            const uint8_t *wbase =
-                (e == p.E ? p.shared : p.routed + (size_t)e * p.expert_bytes) + p.mat_off;
+            const __half *abase = p.aplain + (size_t)rt * kTM * p.K;
             for (int ks = 0; ks < ksteps; ks++, gs++) {
                 const int slot = gs % S;
                 if (gs >= (uint32_t)S &&
@@ -241,44 +257,136 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
                     ok = false;
                     break;
                 }
-                const int seg = ks >> 1, h = ks & 1;
                 uint8_t *sA = stages + slot * SB;
 #pragma unroll
-                for (int m = 0; m < Cfg::kMats; m++) {
-                    const uint8_t *wm = wbase + m * p.mat_bytes;
+                for (int i = 0; i < 8; i++) {
+                    const int idx = dt + 128 * i, r = idx >> 3, ch = idx & 7;
+                    cp_async16(sA + (r >> 3) * 1024 + ch * 128 + (r & 7) * 16,
+                               abase + (size_t)r * p.K + ks * kKS + ch * 8, 16u);
+                }
+                cp_async_commit();
+                if (prev >= 0) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_a[prev]);
+                }
+                prev = slot;
+            }
+        }
+        cp_async_wait<0>();
+        if (prev >= 0 && !*abort_flag) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[prev]);
+        }
+    } else if (kMode != kModePlain && warp < kWarpDq0 + kNumDq) {
+        // ---------------------------------------------------------- dequant
+        const int dt = threadIdx.x - 32 * kWarpDq0;  // 0..127
+        const int L = dt & 31, sl0 = dt >> 5;        // slabs sl0 and sl0 + 4
+        const int g8 = L >> 2, c = L & 3;
+        const __half2 half2_05 = __float2half2_rn(0.5f);
+        // packed words of one stage for this thread: [matrix][slab]
+        struct Raw {
+            uint2 lo[Cfg::kMats][2];
+            uint32_t hi[Cfg::kMats][2];
+            uint2 sc[Cfg::kMats][2];
+        };
+        auto fetch = [&](int t, int ks, Raw &r) {
+            const int rt = t % p.n_rt;
+            const int e = __ldg(&p.units[t / p.n_rt].x);
+            const uint8_t *wbase =
+                (e == p.E ? p.shared : p.routed + (size_t)e * p.expert_bytes) + p.mat_off;
+            const int seg = ks >> 1, h = ks & 1;
 #pragma unroll
-                    for (int si = 0; si < 2; si++) {
-                        const int sl = sl0 + 4 * si;
-                        const uint8_t *un = wm + ((size_t)(rt * 8 + sl) * p.nseg + seg) * UB;
-                        const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
-                        uint32_t hi = 0;
-                        if (kBits == 3)
-                            hi = __ldg(reinterpret_cast<const uint32_t *>(un + kLoBytes + L * 8 + 4 * h));
-                        const uint2 sc =
-                            __ldg(reinterpret_cast<const uint2 *>(un + SOFF + (4 * g8 + 2 * h) * 4));
+            for (int m = 0; m < Cfg::kMats; m++)
 #pragma unroll
-                        for (int bw = 0; bw < 2; bw++) {
-                            const uint32_t lw = bw ? lo.y : lo.x;
-                            const __half2 s2 = __hmul2(u2h(bw ? sc.y : sc.x), half2_05);
-                            const __half2 s_lo = __low2half2(s2), s_hi = __high2half2(s2);
+                for (int si = 0; si < 2; si++) {
+                    const uint8_t *un = wbase + m * p.mat_bytes +
+                                        ((size_t)(rt * 8 + sl0 + 4 * si) * p.nseg + seg) * UB;
+                    r.lo[m][si] = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
+                    r.hi[m][si] = kBits == 3 ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                   un + kLoBytes + L * 8 + 4 * h))
+                                             : 0u;
+                    r.sc[m][si] = __ldg(
+                        reinterpret_cast<const uint2 *>(un + SOFF + (4 * g8 + 2 * h) * 4));
+                }
+        };
+        // Walk the (tile, stage) sequence with three register buffers: the raw
+        // words of position i+3 are requested right after position i is
+        // dequantised, i.e. two stages of work before they are needed.
+        struct Pos {
+            int t, ks;
+        };
+        auto advance = [&](Pos q) {
+            if (++q.ks == ksteps) {
+                q.ks = 0;
+                q.t += gridDim.x;
+            }
+            return q;
+        };
+        uint32_t gs = 0;
+        bool ok = true;
+        // returns false when the pipeline must stop (end of work or abort)
+        auto step = [&](const Raw &cur, Pos q) -> bool {
+            const int slot = gs % S;
+            if (gs >= (uint32_t)S &&
+                !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag))
+                return false;
+            const int h = q.ks & 1;
+            (void)h;
+            uint8_t *sA = stages + slot * SB;
 #pragma unroll
-                            for (int s = 0; s < 2; s++)
+            for (int m = 0; m < Cfg::kMats; m++)
 #pragma unroll
-                                for (int r = 0; r < 4; r++) {
-                                    const uint32_t pr = dq_pair<false, kBits>(lw, hi, 4 * s + r, 8 * bw);
-                                    const __half2 v = __hmul2(u2h(pr), (r & 1) ? s_hi : s_lo);
-                                    const int R8 = 2 * sl + (r & 1);
-                                    const int kc = 4 * bw + 2 * s + (r >> 1);
-                                    *reinterpret_cast<uint32_t *>(sA + m * kTileA + R8 * 1024 +
-                                                                  kc * 128 + g8 * 16 + 4 * c) = h2u(v);
-                                }
-                        }
+                for (int si = 0; si < 2; si++) {
+                    const int sl = sl0 + 4 * si;
+#pragma unroll
+                    for (int bw = 0; bw < 2; bw++) {
+                        const uint32_t lw = bw ? cur.lo[m][si].y : cur.lo[m][si].x;
+                        const __half2 s2 =
+                            __hmul2(u2h(bw ? cur.sc[m][si].y : cur.sc[m][si].x), half2_05);
+                        const __half2 s_lo = __low2half2(s2), s_hi = __high2half2(s2);
+#pragma unroll
+                        for (int s = 0; s < 2; s++)
+#pragma unroll
+                            for (int r = 0; r < 4; r++) {
+                                const uint32_t pr =
+                                    kBits == 2 ? dq2_pair(lw, 4 * s + r)
+                                               : dq_pair<false, kBits>(lw, cur.hi[m][si],
+                                                                       4 * s + r, 8 * bw);
+                                const __half2 v = __hmul2(u2h(pr), (r & 1) ? s_hi : s_lo);
+                                const int R8 = 2 * sl + (r & 1);
+                                const int kc = 4 * bw + 2 * s + (r >> 1);
+                                *reinterpret_cast<uint32_t *>(sA + m * kTileA + R8 * 1024 +
+                                                              kc * 128 + g8 * 16 + 4 * c) = h2u(v);
+                            }
                     }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (L == 0) mbar_arrive(&full_a[slot]);
-            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (L == 0) mbar_arrive(&full_a[slot]);
+            gs++;
+            return true;
+        };
+        Raw r0, r1, r2;
+        Pos p0{(int)blockIdx.x, 0}, p1 = advance(p0), p2 = advance(p1);
+        if (p0.t < n_tiles) fetch(p0.t, p0.ks, r0);
+        if (p1.t < n_tiles) fetch(p1.t, p1.ks, r1);
+        if (p2.t < n_tiles) fetch(p2.t, p2.ks, r2);
+        while (ok) {
+            if (p0.t >= n_tiles || !step(r0, p0)) break;
+            const Pos p3 = advance(p2);
+            if (p3.t < n_tiles) fetch(p3.t, p3.ks, r0);
+            if (p1.t >= n_tiles || !step(r1, p1)) break;
+            const Pos p4 = advance(p3);
+            if (p4.t < n_tiles) fetch(p4.t, p4.ks, r1);
+            if (p2.t >= n_tiles || !step(r2, p2)) break;
+            const Pos p5 = advance(p4);
+            if (p5.t < n_tiles) fetch(p5.t, p5.ks, r2);
+            p0 = p3;
+            p1 = p4;
+            p2 = p5;
         }
     } else {
         // ---------------------------------------------------------- epilogue
@@ -289,7 +397,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
             if (!pipe_wait(acc_full, it & 1, p.budget, p.err, abort_flag)) break;
             tc_fence_after();
             const int rt = t % p.n_rt;
-            const int4 un = p.units[t / p.n_rt];
+            const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
             const int row = rt * kTM + r_in;
             for (int nc = 0; nc < kTN / 32; nc++) {
@@ -307,12 +415,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
                             p.out[(size_t)(slot0 + tok) * p.out_ld + row] = __float2half_rn(a);
                         }
                     }
-                } else {
+                } else if (kMode == kModeDown) {
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
                         const int tok = nc * 32 + j;
                         if (tok < n)
                             p.out[(size_t)(slot0 + tok) * p.out_ld + row] = __float2half_rn(gv[j]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int tok = nc * 32 + j;
+                        if (tok < n) p.out32[(size_t)(slot0 + tok) * p.out_ld + row] = gv[j];
                     }
                 }
             }
@@ -343,7 +457,7 @@ __global__ void to_half_kernel(const __nv_bfloat16 *__restrict__ x, __half *__re
 
 static int g_num_sms = 0;
 
-template <int kBits, bool kGateUp>
+template <int kBits, int kMode>
 static void run_umma(const UmmaParams &p, int max_tiles, cudaStream_t s) {
     if (g_num_sms == 0) {
         int dev = 0;
@@ -352,17 +466,18 @@ static void run_umma(const UmmaParams &p, int max_tiles, cudaStream_t s) {
     }
     int grid = max_tiles < g_num_sms ? max_tiles : g_num_sms;
     if (grid <= 0) return;
-    umma_expert_kernel<kBits, kGateUp>
-        <<<grid, kUmmaThreads, UmmaCfg<kGateUp>::kSmem, s>>>(p);
+    umma_expert_kernel<kBits, kMode><<<grid, kUmmaThreads, UmmaCfg<kMode>::kSmem, s>>>(p);
 }
 
-void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                         const int *n_units, int units_max, const int32_t *list, int Tk,
-                         const void *x, void *x16, void *a, void *Y, int *err, long long budget,
-                         int T, cudaStream_t s) {
-    size_t n8 = (size_t)T * g.H / 8;
+void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s) {
+    size_t n8 = n / 8;
     to_half_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
         reinterpret_cast<const __nv_bfloat16 *>(x), reinterpret_cast<__half *>(x16), n8);
+}
+
+static UmmaParams base_params(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                              const int *n_units, const int32_t *list, int Tk, int *err,
+                              long long budget) {
     UmmaParams p{};
     p.routed = w.routed;
     p.shared = w.shared;
@@ -375,7 +490,14 @@ void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *
     p.Tk = Tk;
     p.err = err;
     p.budget = budget;
-    // gate/up: A = Wg, Wu (Ip rows, K = H); B = x rows gathered by token
+    return p;
+}
+
+void launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                        const int *n_units, int units_max, const int32_t *list, int Tk,
+                        const void *x16, void *a, int *err, long long budget, cudaStream_t s) {
+    // A = Wg, Wu (Ip rows, K = H); B = x rows (fp16 copy) gathered by token
+    UmmaParams p = base_params(g, w, units, n_units, list, Tk, err, budget);
     p.mat_off = 0;
     p.xin = reinterpret_cast<const __half *>(x16);
     p.K = g.H;
@@ -384,10 +506,16 @@ void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *
     p.out = reinterpret_cast<__half *>(a);
     p.out_ld = g.Ip;
     if (g.bits == 2)
-        run_umma<2, true>(p, units_max * p.n_rt, s);
+        run_umma<2, kModeGateUp>(p, units_max * p.n_rt, s);
     else
-        run_umma<3, true>(p, units_max * p.n_rt, s);
-    // down: A = Wd (H rows, K = Ip); B = a rows by slot
+        run_umma<3, kModeGateUp>(p, units_max * p.n_rt, s);
+}
+
+void launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                      const int *n_units, int units_max, const void *a, void *Y, int *err,
+                      long long budget, cudaStream_t s) {
+    // A = Wd (H rows, K = Ip); B = a rows by slot
+    UmmaParams p = base_params(g, w, units, n_units, nullptr, 0, err, budget);
     p.mat_off = 2 * g.mat_bytes;
     p.xin = reinterpret_cast<const __half *>(a);
     p.K = g.Ip;
@@ -396,17 +524,38 @@ void launch_umma_experts(const Geometry &g, const ExpertWeights &w, const int4 *
     p.out = reinterpret_cast<__half *>(Y);
     p.out_ld = g.H;
     if (g.bits == 2)
-        run_umma<2, false>(p, units_max * p.n_rt, s);
+        run_umma<2, kModeDown>(p, units_max * p.n_rt, s);
     else
-        run_umma<3, false>(p, units_max * p.n_rt, s);
+        run_umma<3, kModeDown>(p, units_max * p.n_rt, s);
+}
+
+void launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
+                       int *err, long long budget, cudaStream_t s) {
+    UmmaParams p{};
+    p.aplain = A;
+    p.xin = x16;
+    p.direct_T = T;
+    p.K = K;
+    p.nseg = K / kSegCols;
+    p.n_rt = rows / kTM;
+    p.out32 = D;
+    p.out_ld = rows;
+    p.err = err;
+    p.budget = budget;
+    run_umma<2, kModePlain>(p, ((T + kTN - 1) / kTN) * p.n_rt, s);
 }
 
 cudaError_t umma_init_attributes(int max_smem) {
     cudaError_t e;
-    if ((e = allow_max_dyn_smem(umma_expert_kernel<2, true>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(umma_expert_kernel<3, true>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(umma_expert_kernel<2, false>, max_smem)) != cudaSuccess) return e;
-    return allow_max_dyn_smem(umma_expert_kernel<3, false>, max_smem);
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<2, kModeGateUp>, max_smem)) != cudaSuccess)
+        return e;
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<3, kModeGateUp>, max_smem)) != cudaSuccess)
+        return e;
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<2, kModeDown>, max_smem)) != cudaSuccess)
+        return e;
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<3, kModeDown>, max_smem)) != cudaSuccess)
+        return e;
+    return allow_max_dyn_smem(umma_expert_kernel<2, kModePlain>, max_smem);
 }
 
 }  // namespace strata

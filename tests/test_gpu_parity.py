@@ -219,3 +219,37 @@ def test_rmsnorm_bit_exact():
     qe.strata_moe_rmsnorm(xt.data_ptr(), out.data_ptr(), 37, 2560, None)
     torch.cuda.synchronize()
     assert np.array_equal(from_dev_bf16(out), oracle.rmsnorm(x))
+
+
+def _route_case(layer, T, seed, label):
+    L = qe.Layer(layer, max_tokens=T)
+    x = gen.hidden(T, layer.shape.hidden, seed=seed)
+    check_route(L, layer, x, T, label)
+
+
+@pytest.mark.parametrize("T", [300, 1000], ids=["T300", "T1000"])
+def test_screened_router_ties_and_near_ties(T):
+    """Above 256 tokens the router screens on the tensor cores and recomputes
+    candidates exactly; picks must still be the oracle's bit for bit when logits
+    tie exactly (duplicated router rows, lower id first), when every logit ties
+    (zero router: all experts are candidates) and when rows differ by one ulp."""
+    import copy
+    shape = gen.LayerShape(hidden=256, n_experts=512, top_k=10, inter=64, bits=2,
+                           router_bias=True)
+    base = gen.layer_weights(shape, seed=31)
+    dup = copy.copy(base)
+    W = base.router_w.copy()
+    W[1::2] = W[0::2]
+    b = base.router_b.copy()
+    b[1::2] = b[0::2]
+    dup.router_w, dup.router_b = W, b
+    _route_case(dup, T, 5, "duplicated rows")
+    near = copy.copy(base)
+    W2 = base.router_w.copy()
+    W2[1::2] = np.nextafter(W2[0::2], np.float32(np.inf))
+    near.router_w, near.router_b = W2, b
+    _route_case(near, T, 6, "one-ulp rows")
+    zero = copy.copy(base)
+    zero.router_w = np.zeros_like(base.router_w)
+    zero.router_b = np.zeros_like(base.router_b)
+    _route_case(zero, T, 7, "zero router")
