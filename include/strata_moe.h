@@ -174,7 +174,11 @@ strata_status strata_moe_debug_dequant(strata_moe_t h, int expert, int mat, int 
 
 /* Options (strata_moe_set_option). */
 enum {
-    STRATA_OPT_PATH = 1,        /* 0 auto (default), 1 force decode GEMV, 2 force prefill GEMM */
+    STRATA_OPT_PATH = 1,        /* 0 auto (default: T <= DECODE_MAX_T runs the fused decode
+                                   kernel where it applies, else the decode GEMV chain; larger T
+                                   the prefill GEMM), 1 force the decode GEMV kernel chain,
+                                   2 force the prefill GEMM, 3 force the fused decode kernel
+                                   (T <= 64, E <= 512; forward fails otherwise) */
     STRATA_OPT_WAIT_BUDGET = 2, /* bound of every device-side wait, in SM clock cycles
                                    (default 4e9); 0 makes every wait give up at once */
     STRATA_OPT_DECODE_MAX_T = 3 /* largest T run by the decode kernels in auto mode (default 64) */

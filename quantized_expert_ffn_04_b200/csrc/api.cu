@@ -81,8 +81,13 @@ struct strata_moe {
     void *Y = nullptr;            // fp32 (decode) / fp16 (prefill) [slots][H]
     int *err = nullptr;
     void *xio = nullptr, *yio = nullptr, *xn = nullptr;  // bf16 [max_tokens][H]
-    void *x16 = nullptr;                                 // fp16 [max_tokens][H]
+    // fp16 token operand of the tensor-core path, [max_tokens * k + max_tokens][H]:
+    // routed token rows in slot order, then (at row T * k) the fp16 copy of x
+    void *xs = nullptr;
     float *dsplit = nullptr;  // [max_tokens][router_rows] screening GEMM output (T > 256)
+    // fused decode counters: [units (tile 8)] then [max_tokens][H / 128]
+    int *fused_cnt = nullptr;
+    int *tok_groups = nullptr;  // router top-k counters (one per token group, self-resetting)
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
     // options
     int path = 0;
@@ -163,8 +168,10 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->xio = take(T * H * 2);
     h->yio = take(T * H * 2);
     h->xn = take(T * H * 2);
-    h->x16 = take(T * H * 2);
+    h->xs = take(slots * H * 2);
     h->dsplit = (float *)take(T > (size_t)kSmallMaxT ? T * (size_t)h->router_rows * 4 : 0);
+    h->fused_cnt = (int *)take(((size_t)units + T * (H / 128)) * 4);
+    h->tok_groups = (int *)take(64 * 4);
     return off;
 }
 
@@ -212,6 +219,11 @@ void probe(strata_moe_t h, int stage, bool begin, cudaStream_t s) {
         cudaEventRecord(e, s);
 }
 
+// The fp16 copy of x inside the token operand (after the T * k routed rows).
+__half *x16_of(strata_moe_t h, int T) {
+    return reinterpret_cast<__half *>(h->xs) + (size_t)T * h->geo.k * h->geo.H;
+}
+
 // Router + top-k + dispatch into the handle's workspace.  Above kSmallMaxT
 // tokens the router runs on the tensor cores (screening GEMM on the fp16 copy
 // of x, which the prefill experts reuse) followed by the exact recompute of
@@ -220,9 +232,11 @@ strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStre
     const Geometry &g = h->geo;
     probe(h, kStRouter, true, s);
     if (T > kSmallMaxT) {
-        launch_to_half(x, h->x16, (size_t)T * g.H, s);
-        launch_umma_plain(h->router_split, h->router_rows, (const __half *)h->x16, T, g.H,
-                          h->dsplit, h->err, h->budget, s);
+        launch_to_half(x, x16_of(h, T), (size_t)T * g.H, s);
+        cudaError_t ce = launch_umma_plain(h->router_split, h->router_rows, x16_of(h, T), T,
+                                           g.H, h->dsplit, h->err, h->budget, s);
+        if (ce != cudaSuccess)
+            return fail(STRATA_ERR_CUDA, "router screening GEMM: %s", cudaGetErrorString(ce));
         launch_screen_topk(h->dsplit, h->router_rows, x, T, g.H, h->router_wp, h->router_b, g.E,
                            g.k, h->screen_gam, h->screen_wmax, h->screen_bmax, h->idx, h->wts, s);
     } else {
@@ -245,13 +259,43 @@ strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStre
 }
 
 bool use_decode_path(strata_moe_t h, int T) {
-    if (h->path == 1) return true;
+    if (h->path == 1 || h->path == 3) return true;
     if (h->path == 2) return false;
     return T <= h->decode_max_t;
 }
 
+// The fused decode kernel: forced (path 3), or in auto mode for every decode
+// batch it supports.
+bool use_fused_path(strata_moe_t h, int T) {
+    if (h->path == 3) return true;
+    return h->path == 0 && T <= h->decode_max_t && fused_decode_supported(h->geo, T);
+}
+
+// Router (+ fp16 copy of x and zeroed counters), then the fused kernel.
+strata_status run_forward_fused(strata_moe_t h, const void *x, int T, void *y, bool residual,
+                                cudaStream_t s) {
+    const Geometry &g = h->geo;
+    if (!fused_decode_supported(g, T))
+        return fail(STRATA_ERR_INVALID_ARG, "the fused decode kernel does not support T=%d", T);
+    const int umax = max_units(T, g.k, g.E, 8);
+    probe(h, kStRouter, true, s);
+    launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s, x16_of(h, T),
+                  h->fused_cnt, umax + T * (g.H / 128), g.k, h->idx, h->wts, h->tok_groups);
+    probe(h, kStRouter, false, s);
+    ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
+    probe(h, kStGateUp, true, s);
+    cudaError_t ce = launch_fused_decode(g, w, h->idx, h->wts, x16_of(h, T), T, umax, h->a,
+                                         (float *)h->Y, y, residual, h->fused_cnt,
+                                         h->fused_cnt + umax, h->err, h->budget, s);
+    probe(h, kStGateUp, false, s);
+    if (ce != cudaSuccess)
+        return fail(STRATA_ERR_CUDA, "fused decode kernel: %s", cudaGetErrorString(ce));
+    return check_launch("fused decode kernels");
+}
+
 strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool residual,
                           cudaStream_t s) {
+    if (use_fused_path(h, T)) return run_forward_fused(h, x, T, y, residual, s);
     const Geometry &g = h->geo;
     const bool decode = use_decode_path(h, T);
     const int tile = decode ? 8 : kUmmaTile;
@@ -272,12 +316,18 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
         // the gate/up probe brackets the gate/up GEMM (and, for T <= kSmallMaxT,
         // the fp16 token copy, which larger batches make in the router stage)
         probe(h, kStGateUp, true, s);
-        if (T <= kSmallMaxT) launch_to_half(x, h->x16, (size_t)T * g.H, s);
-        launch_umma_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, h->x16, h->a,
-                           h->err, h->budget, s);
+        if (T <= kSmallMaxT) launch_to_half(x, x16_of(h, T), (size_t)T * g.H, s);
+        launch_gather_rows(h->list, T * g.k, x16_of(h, T), h->xs, g.H, s);
+        cudaError_t ce = launch_umma_gateup(g, w, h->units, h->n_units, umax, T * g.k + T, h->xs,
+                                            h->a, h->err, h->budget, s);
+        if (ce != cudaSuccess)
+            return fail(STRATA_ERR_CUDA, "gate/up GEMM: %s", cudaGetErrorString(ce));
         probe(h, kStGateUp, false, s);
         probe(h, kStDown, true, s);
-        launch_umma_down(g, w, h->units, h->n_units, umax, h->a, h->Y, h->err, h->budget, s);
+        ce = launch_umma_down(g, w, h->units, h->n_units, umax, T * g.k + T, h->a, h->Y, h->err,
+                              h->budget, s);
+        if (ce != cudaSuccess)
+            return fail(STRATA_ERR_CUDA, "down GEMM: %s", cudaGetErrorString(ce));
         probe(h, kStDown, false, s);
     }
     probe(h, kStCombine, true, s);
@@ -309,11 +359,12 @@ int strata_moe_launch_count(strata_moe_t h, int T) {
     if (T == 0) return 0;
     // up to kSmallMaxT tokens: router, fused top-k + dispatch; above: fp16 token
     // copy, screening GEMM, screened top-k, 3 dispatch kernels.  Then gate/up +
-    // down (+ the fp16 token copy on the prefill path when T <= kSmallMaxT),
-    // and the combine.
+    // down (the tensor-core path adds the slot-order row gather, and the fp16
+    // token copy when T <= kSmallMaxT), and the combine.
+    if (use_fused_path(h, T)) return 2;  // router, fused layer kernel
     const bool decode = use_decode_path(h, T);
-    if (T <= kSmallMaxT) return 2 + (decode ? 2 : 3) + 1;
-    return 6 + 2 + 1;
+    if (T <= kSmallMaxT) return 2 + (decode ? 2 : 4) + 1;
+    return 6 + 3 + 1;
 }
 
 strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_weights *wts,
@@ -470,7 +521,8 @@ strata_status strata_moe_set_option(strata_moe_t h, int option, int64_t value) {
     if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
     switch (option) {
     case STRATA_OPT_PATH:
-        if (value < 0 || value > 2) return fail(STRATA_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+        if (value < 0 || value > 3)
+            return fail(STRATA_ERR_INVALID_ARG, "path must be 0, 1, 2 or 3");
         h->path = (int)value;
         return STRATA_OK;
     case STRATA_OPT_WAIT_BUDGET:

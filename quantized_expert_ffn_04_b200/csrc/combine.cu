@@ -164,6 +164,7 @@ cudaError_t init_kernel_attributes() {
     if ((e = route_init_attributes(max_smem)) != cudaSuccess) return e;
     if ((e = gemv_init_attributes(max_smem)) != cudaSuccess) return e;
     if ((e = umma_init_attributes(max_smem)) != cudaSuccess) return e;
+    if ((e = fused_init_attributes(max_smem)) != cudaSuccess) return e;
     if (dev < 64) done[dev] = true;
     return cudaSuccess;
 }

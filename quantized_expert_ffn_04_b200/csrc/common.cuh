@@ -91,20 +91,18 @@ STRATA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// As mbar_try_wait, but the thread may sleep in hardware for up to `hint_ns`
-// nanoseconds waiting for the phase (instead of spinning on issue slots).
-STRATA_DEV bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+// Non-blocking test of phase `parity` (never suspends the thread).
+STRATA_DEV bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
-constexpr uint32_t kSleepHintNs = 100000;  // re-check the wait budget every 0.1 ms
 
 // Wait for phase `parity` of `bar`, giving up after `budget` SM cycles.  On
 // give-up the handle's error word gets kErrTimeout and false is returned.
@@ -114,7 +112,7 @@ STRATA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget, int 
         return false;
     }
     long long t0 = clock64();
-    while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
+    while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > budget) {
             if (err) atomicCAS(err, 0, kErrTimeout);
             return false;
@@ -313,6 +311,34 @@ STRATA_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of
+// 128 bytes (64 fp16 of K), 8-row groups 1024 bytes apart, the group base
+// 1024-byte aligned.  Steps along K inside the 128-byte row add to the start
+// address (the swizzle is a function of the address bits).
+STRATA_DEV uint64_t umma_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3fff);
+    d |= (uint64_t)1 << 16;              // leading offset: not used by swizzled K-major
+    d |= (uint64_t)(1024 >> 4) << 32;    // 8-row groups
+    d |= (uint64_t)1 << 46;              // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;              // 128-byte swizzle
+    return d;
+}
+
+// Tensor-map (TMA) loads into this CTA's shared memory, completing bytes on
+// `bar`; no multicast.  `map` is the generic address of a CUtensorMap kernel
+// parameter; x (the column) must make x * 2 bytes a multiple of 16.
+STRATA_DEV void tma_load_2d(void *dst, const void *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+STRATA_DEV void prefetch_tmap(const void *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
 // 16-byte cp.async global -> shared; bytes beyond `src_bytes` (0 or 16) are zero.
 STRATA_DEV void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
@@ -361,7 +387,9 @@ STRATA_DEV uint32_t dq2_pair(uint32_t w, int rp) {
 // one asm block so they land directly in the operand registers.
 STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, uint32_t b2,
                            uint32_t b3) {
-    asm volatile(
+    // pure register arithmetic (not volatile): the compiler may schedule the
+    // blocks of a loop around one another
+    asm(
         "{\n\t"
         ".reg .b32 s8, s2, h0, h1, h2, h3, h4, h5, h6, h7;\n\t"
         ".reg .f32 z;\n\t"
@@ -393,6 +421,26 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
         : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(0x38003800u), "r"(0x30003000u),
           "r"(0x28002800u), "r"(0x20002000u), "r"(0xE006E006u), "r"(0xD818D818u),
           "r"(0xD060D060u), "r"(0xC980C980u));
+}
+
+// ---------------------------------------------------------------- GEMV blocks
+STRATA_DEV uint32_t comp4(const uint4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// One 32-wide block: D = A_blk(16x32) * B(32x8) with A the exact integers,
+// two mma k-steps.  lo/hi: the lane's code words for this block.
+template <int kBits>
+STRATA_DEV void block_mma(float (&d)[4], uint32_t lo, uint32_t hi, int hshift, uint32_t b0,
+                          uint32_t b1, uint32_t b2, uint32_t b3) {
+    uint32_t a[4];
+    const float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, r, hshift);
+    mma_f16(d, a, b0, b1, z);
+#pragma unroll
+    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, 4 + r, hshift);
+    mma_f16(d, a, b2, b3, d);
 }
 
 }  // namespace strata

@@ -28,25 +28,6 @@ namespace strata {
 
 constexpr int kTile = 8;  // tokens per unit (mma N)
 
-__device__ __forceinline__ uint32_t comp4(const uint4 &v, int i) {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
-// One 32-wide block: D = A_blk(16x32) * B(32x8) with A the exact integers,
-// two mma k-steps.  lo/hi: the lane's code words for this block.
-template <int kBits>
-__device__ __forceinline__ void block_mma(float (&d)[4], uint32_t lo, uint32_t hi, int hshift,
-                                          uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-    uint32_t a[4];
-    const float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, r, hshift);
-    mma_f16(d, a, b0, b1, z);
-#pragma unroll
-    for (int r = 0; r < 4; r++) a[r] = dq_pair<false, kBits>(lo, hi, 4 + r, hshift);
-    mma_f16(d, a, b2, b3, d);
-}
-
 // Accumulate one 16 x (ns*128) slab of a matrix whose units sit in smem at
 // `w` against the fp16 token rows staged at `xb` (row pitch `pitch` elements,
 // `xrows` rows staged; the other mma columns read row 0 and are ignored).

@@ -29,8 +29,14 @@ void launch_debug_dequant(const uint8_t *mat, int bits, int Kp, int row0, int nr
 
 // ---- route.cu
 // Router weight in the lane-interleaved layout: Wp[e][H/128][32 lanes][4].
+// For the fused decode kernel that follows (all optional): x16, the fp16 copy
+// of x [T][H]; zero, nzero ints zeroed; tok_done (one counter per group of up
+// to 8 tokens, zero between launches): the top-k of every token written to
+// idx / w [T][k] by the last CTA of its token group.
 void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                   float *logits, cudaStream_t s);
+                   float *logits, cudaStream_t s, void *x16 = nullptr, int *zero = nullptr,
+                   int nzero = 0, int k = 0, int32_t *idx = nullptr, float *w = nullptr,
+                   int *tok_done = nullptr);
 void launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
                  cudaStream_t s);
 
@@ -79,19 +85,38 @@ void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *uni
 // ---- umma.cu (prefill)
 // x (bf16) -> x16 (fp16 copy), then gate/up (a: fp16 [slots][Ip]) and down
 // (Y: fp16 [slots][H]) on the tensor cores.  Units of up to 256 tokens.
+// The token operand xs is fp16 [slots][H] with slots = Tk + T: the routed
+// rows in slot order (launch_gather_rows), then the fp16 copy of x; a holds
+// `slots` rows too.  Each returns the launch status (an error also when the
+// tensor maps cannot be encoded).
 constexpr int kUmmaTile = 256;
-void launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                        const int *n_units, int units_max, const int32_t *list, int Tk,
-                        const void *x16, void *a, int *err, long long budget, cudaStream_t s);
-void launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                      const int *n_units, int units_max, const void *a, void *Y, int *err,
-                      long long budget, cudaStream_t s);
+void launch_gather_rows(const int32_t *list, int Tk, const void *x16, void *xs, int H,
+                        cudaStream_t s);
+cudaError_t launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                               const int *n_units, int units_max, int slots, const void *xs,
+                               void *a, int *err, long long budget, cudaStream_t s);
+cudaError_t launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                             const int *n_units, int units_max, int slots, const void *a, void *Y,
+                             int *err, long long budget, cudaStream_t s);
 // Plain fp16 GEMM on the tensor cores: D[t][r] = sum_k x16[t][k] * A[r][k],
 // rows a multiple of 128, K a multiple of 128; fp32 out with row stride `rows`.
-void launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
-                       int *err, long long budget, cudaStream_t s);
+cudaError_t launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
+                              int *err, long long budget, cudaStream_t s);
 void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s);
 cudaError_t umma_init_attributes(int max_smem);
+
+// ---- decode.cu (fused decode layer, T <= 64)
+// After launch_router(..., x16, counters, units_max + T (H / 128), k, idx, w,
+// tok_done): dispatch, gate/up, down and combine in one kernel (programmatic
+// dependent launch).
+// done_gu [units_max] and done_tok [T][H / 128] are the router-zeroed counters.
+int fused_decode_supported(const Geometry &g, int T);
+cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const int32_t *idx,
+                                const float *wts, const void *x16, int T, int units_max, void *a,
+                                float *Y,
+                                void *out, bool residual, int *done_gu, int *done_tok, int *err,
+                                long long budget, cudaStream_t s);
+cudaError_t fused_init_attributes(int max_smem);
 
 // ---- combine.cu
 // out[t] = Y[Tk + t] + sum_j (ascending expert id) w[t][j] * Y[slot[t][j]]; bf16.

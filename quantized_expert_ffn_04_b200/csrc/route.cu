@@ -21,19 +21,123 @@
 
 namespace strata {
 
+// ============================================================== warp top-k
+// Order-preserving 32-bit key of a logit: larger float <=> larger key; -0 is
+// read as +0 (equal floats, equal keys) and a NaN as -inf (it ranks last).
+// Key 0 is below every logit and marks a taken or missing entry.
+__device__ __forceinline__ uint32_t logit_key(float f) {
+    if (f != f) f = -INFINITY;
+    if (f == 0.0f) f = 0.0f;
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-k of one token by one warp (E <= 512: lane l holds logits l, l+32, ...).
+// Each round takes the largest key over the warp (redux.sync max) and, among
+// the lanes holding it, the lowest expert id (redux.sync min), i.e. the larger
+// logit and on equal logits the lower id; the winning lane drops that entry.
+// Lane j < k ends with pick j and its weight exp(l_j - m) / sum.
+__device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
+                                        int &pick_e, float &pick_w) {
+    uint32_t key[16];
+    const int nq = (E + 31) >> 5;
+#pragma unroll
+    for (int q = 0; q < 16; q++) {
+        const int e = q * 32 + lane;
+        key[q] = (q < nq && e < E) ? logit_key(__ldcg(row + e)) : 0u;
+    }
+    // this lane's best entry: largest key, then lowest q (= lowest id)
+    uint32_t bk = 0u;
+    int bq = 0;
+#pragma unroll
+    for (int q = 15; q >= 0; q--) {
+        const bool t = key[q] >= bk && key[q] != 0u;
+        bk = t ? key[q] : bk;
+        bq = t ? q : bq;
+    }
+    uint32_t my_k = 0u;
+    int my_e = -1;
+    for (int j = 0; j < k; j++) {
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == wk && bk != 0u) ? (uint32_t)(bq * 32 + lane) : 0xffffffffu;
+        const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
+        if (lane == j) {
+            my_k = wk;
+            my_e = (int)we;
+        }
+        // the winning lane drops the entry and finds its next best
+        const bool mine = (int)(we & 31u) == lane;
+        const int wq = (int)(we >> 5);
+        uint32_t nk = 0u;
+        int nb = 0;
+#pragma unroll
+        for (int q = 15; q >= 0; q--) {
+            key[q] = (mine && q == wq) ? 0u : key[q];
+            const bool t = key[q] >= nk && key[q] != 0u;
+            nk = t ? key[q] : nk;
+            nb = t ? q : nb;
+        }
+        bk = mine ? nk : bk;
+        bq = mine ? nb : bq;
+    }
+    const float my_v = key_logit(my_k);
+    const float m = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = lane < k ? expf(my_v - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    pick_e = my_e;
+    pick_w = ex / sum;
+}
+
 // ============================================================== router
 // CTA: 4 warps; warp owns EE experts, lanes are the 32 residue classes of the
 // fixed order; TT tokens per CTA staged in smem as fp32 in the same
 // lane-interleaved layout as the weights: xs[tt][s4][lane] = float4 of
 // x[128*s4 + 32*j + lane], j = 0..3.
+// Optional side outputs for the fused decode kernel that follows: x16 (fp16
+// copy of x, written by the CTAs of expert block 0), nzero ints zeroed, and
+// the top-k picks: with tok_done set, the last CTA to finish a token group
+// (a counter per group, reset by that CTA) runs the top-k of its tokens and
+// writes idx / wout, so the next kernel reads T k picks, not T E logits.
 template <int TT, int EE, int CH>
 __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__restrict__ x, int T,
                                                      int H, const float4 *__restrict__ Wp,
                                                      const float *__restrict__ bias, int E,
-                                                     float *__restrict__ logits) {
+                                                     float *__restrict__ logits,
+                                                     __half *__restrict__ x16,
+                                                     int *__restrict__ zero, int nzero, int k,
+                                                     int32_t *__restrict__ idx,
+                                                     float *__restrict__ wout,
+                                                     int *__restrict__ tok_done) {
     extern __shared__ float4 xs[];
+    // a dependent kernel may be scheduled now; it waits for this grid's
+    // completion before reading anything written here
+    grid_launch_dependents();
     const int ns4 = H / 128;
     const int t0 = blockIdx.y * TT;
+    if (zero && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
+    const bool write16 = x16 != nullptr && blockIdx.x == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = (blockIdx.x * 4 + warp) * EE;
+    // the first CH steps of this warp's weights are requested before the
+    // token rows are staged, so the two latencies overlap
+    float4 wv[CH][EE];
+    auto load_w = [&](int s0) {
+#pragma unroll
+        for (int c = 0; c < CH; c++)
+#pragma unroll
+            for (int b = 0; b < EE; b++) {
+                int e = e0 + b, s4 = s0 + c;
+                wv[c][b] = (e < E && s4 < ns4) ? __ldg(Wp + ((size_t)e * ns4 + s4) * 32 + lane)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+    };
+    load_w(0);
     // stage TT token rows (16 bytes = 8 bf16 per chunk); each thread requests a
     // batch of 8 chunks before storing any, so the loads overlap
     const int nchunk = TT * H / 8;
@@ -55,6 +159,15 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
             if (idx >= nchunk) break;
             const int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
             const __nv_bfloat16 *pv = reinterpret_cast<const __nv_bfloat16 *>(&v[b]);
+            if (write16 && t0 + tt < T) {
+                uint4 o;
+                __half2 *h2 = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+                for (int q = 0; q < 4; q++)
+                    h2[q] = __floats2half2_rn(__bfloat162float(pv[2 * q]),
+                                              __bfloat162float(pv[2 * q + 1]));
+                *reinterpret_cast<uint4 *>(x16 + (size_t)(t0 + tt) * H + i0) = o;
+            }
 #pragma unroll
             for (int q = 0; q < 8; q++) {
                 const int i = i0 + q;
@@ -64,9 +177,7 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
         }
     }
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e0 = (blockIdx.x * 4 + warp) * EE;
-    if (e0 >= E) return;
+    if (e0 < E) {
     float acc[TT][EE];
 #pragma unroll
     for (int a = 0; a < TT; a++)
@@ -76,15 +187,7 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
     // CH steps of weights are requested before any of them is used, so a warp
     // keeps CH x EE x 512 bytes in flight.
     for (int s0 = 0; s0 < ns4; s0 += CH) {
-        float4 wv[CH][EE];
-#pragma unroll
-        for (int c = 0; c < CH; c++)
-#pragma unroll
-            for (int b = 0; b < EE; b++) {
-                int e = e0 + b, s4 = s0 + c;
-                wv[c][b] = (e < E && s4 < ns4) ? __ldg(Wp + ((size_t)e * ns4 + s4) * 32 + lane)
-                                               : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        if (s0 > 0) load_w(s0);
 #pragma unroll
         for (int c = 0; c < CH; c++) {
             const int s4 = s0 + c;
@@ -124,28 +227,53 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
             }
         }
     }
+    }
+    if (tok_done == nullptr) return;
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(tok_done + blockIdx.y, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();  // every CTA's logits of this token group are visible
+    for (int a = warp; a < TT; a += 4) {
+        const int t = t0 + a;
+        if (t >= T) break;
+        int pe;
+        float pw;
+        warp_topk(logits + (size_t)t * E, E, k, lane, pe, pw);
+        if (lane < k) {
+            idx[(size_t)t * k + lane] = pe;
+            wout[(size_t)t * k + lane] = pw;
+        }
+    }
+    if (threadIdx.x == 0) tok_done[blockIdx.y] = 0;  // ready for the next launch
 }
 
 template <int TT, int EE, int CH>
 static void run_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                       float *logits, cudaStream_t s) {
+                       float *logits, void *x16, int *zero, int nzero, int k, int32_t *idx,
+                       float *w, int *tok_done, cudaStream_t s) {
     size_t smem = (size_t)TT * H * sizeof(float);
     auto kern = router_kernel<TT, EE, CH>;
     dim3 grid((E + 4 * EE - 1) / (4 * EE), (T + TT - 1) / TT);
     kern<<<grid, 128, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
-                                 reinterpret_cast<const float4 *>(Wp), bias, E, logits);
+                                 reinterpret_cast<const float4 *>(Wp), bias, E, logits,
+                                 reinterpret_cast<__half *>(x16), zero, nzero, k, idx, w,
+                                 tok_done);
 }
 
 void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                   float *logits, cudaStream_t s) {
+                   float *logits, cudaStream_t s, void *x16, int *zero, int nzero, int k,
+                   int32_t *idx, float *w, int *tok_done) {
     if (T <= 1)
-        run_router<1, 1, 20>(x, T, H, Wp, bias, E, logits, s);
+        run_router<1, 1, 20>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 4)
-        run_router<4, 1, 20>(x, T, H, Wp, bias, E, logits, s);
+        run_router<4, 1, 20>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 64)
-        run_router<8, 2, 8>(x, T, H, Wp, bias, E, logits, s);
+        run_router<8, 2, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else
-        run_router<8, 8, 2>(x, T, H, Wp, bias, E, logits, s);
+        run_router<8, 8, 2>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
 }
 
 // ============================================================== top-k

@@ -9,21 +9,32 @@
 //
 // Tile: 128 weight rows (MMA M) x up to 256 tokens of one expert (MMA N =
 // the tile's token count rounded up to 16, so a cold expert's short tile does
-// not pay for empty columns), K in stages of 64.  Operands are fp16, K-major, without swizzle, in 8-row x
+// not pay for empty columns), K in stages of 64.  Operands are fp16, K-major.
+// The token operand B is brought in by the tensor memory accelerator with the
+// 128-byte swizzle, 16 consecutive rows per box: gate/up reads the fp16 token
+// rows in slot order (each expert's tokens contiguous, built once per forward
+// by gather_rows_kernel), down reads a by slot, the plain GEMM reads x.  The weight
+// operand A is written by the dequant warps without swizzle, in 8-row x
 // 16-byte core matrices (K-adjacent core matrices 128 B apart, row groups
-// 1024 B apart).  Warp roles:
+// 1024 B apart); the plain GEMM loads A by tensor map as well.  Warp roles:
 //   warp 0      allocates tensor memory; lane 0 issues the MMAs and commits
 //               them to the stage and accumulator barriers;
-//   warp 1      gathers the tile's token rows (fp16) with cp.async;
+//   warp 1      lane 0 issues the tensor-map loads of each stage;
 //   warps 2..5  dequantise the weight tile into the A operand: codes -> exact
-//               odd integers (shift, mask/or against a magic exponent, packed
-//               subtract) -> one packed multiply by d/2, i.e. the fp16 value of
-//               d*(q-c) rounded once to nearest even;
+//               odd integers -> one packed multiply by d/2, i.e. the fp16 value
+//               of d*(q-c) rounded once to nearest even;
 //   warps 6..9  read the accumulators back (tcgen05.ld) and write
-//               a = silu(g) u (gate/up) or y (down) as fp16.
+//               a = silu(g) u (gate/up), y (down) as fp16, or D (plain) as fp32.
+// Down and plain keep two accumulators in tensor memory, so the epilogue of a
+// tile overlaps the MMAs of the next; gate/up uses both halves for g and u.
 // Every wait is bounded; a wait that gives up sets the handle's error word
 // and an abort flag that releases the other roles, and the CTA lets its
 // copies and MMAs land before it frees tensor memory and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,15 +42,16 @@ namespace strata {
 
 constexpr int kTM = 128;                // weight rows per tile
 constexpr int kTN = 256;                // most tokens per tile
-constexpr int kKS = 64;                 // K per stage
+constexpr int kKS = 64;                 // K per stage (one 128-byte swizzle row)
 constexpr int kTileA = kTM * kKS * 2;   // 16 KB
 constexpr int kTileB = kTN * kKS * 2;   // 32 KB
-constexpr int kWarpMma = 0, kWarpLoadB = 1, kWarpDq0 = 2, kNumDq = 4, kNumEpi = 4;  // epilogue: warps 6..9
+constexpr int kBoxRows = 16;            // rows per 2-D box of the token operand
+constexpr int kWarpMma = 0, kWarpLoad = 1, kWarpDq0 = 2, kNumDq = 4, kWarpEpi0 = 6, kNumEpi = 4;
 constexpr int kUmmaThreads = 32 * 10;
 
 // Modes: gate/up (A = dequantised Wg and Wu, SwiGLU epilogue, fp16 out),
-// down (A = dequantised Wd, fp16 out), plain (A = an fp16 matrix copied with
-// cp.async, fp32 out; used by the router's screening GEMM).
+// down (A = dequantised Wd, fp16 out), plain (A = an fp16 matrix loaded by
+// tensor map, fp32 out; used by the router's screening GEMM).
 constexpr int kModeGateUp = 0, kModeDown = 1, kModePlain = 2;
 
 template <int kMode>
@@ -47,11 +59,15 @@ struct UmmaCfg {
     static constexpr int kMats = kMode == kModeGateUp ? 2 : 1;
     static constexpr int kStages = kMode == kModeGateUp ? 3 : 4;
     static constexpr int kStageBytes = kMats * kTileA + kTileB;
-    static constexpr int kTmemCols = kMode == kModeGateUp ? 512 : 256;
-    static constexpr int kSmem = kStages * kStageBytes + 2048;
+    static constexpr int kAccBufs = kMode == kModeGateUp ? 1 : 2;
+    static constexpr int kTmemCols = 512;
+    // stages + alignment slack (1024) + barriers
+    static constexpr int kSmem = kStages * kStageBytes + 1024 + 2048;
 };
 
 struct UmmaParams {
+    CUtensorMap tm_b;   // token operand (see the file comment)
+    CUtensorMap tm_a;   // plain: A [n_rt * 128][K] fp16, boxes of 64 x 128
     const uint8_t *routed;
     const uint8_t *shared;
     size_t expert_bytes, mat_bytes, mat_off;
@@ -60,11 +76,9 @@ struct UmmaParams {
     int E;
     const int32_t *list;
     int Tk;
-    const __half *xin;  // gate/up: x as fp16 [T][K]; down: a [slots][K]; plain: x [T][K]
     int K, nseg, n_rt;
     __half *out;        // gate/up: a [slots][Ip]; down: Y [slots][H]
     float *out32;       // plain: D [T][n_rt * 128]
-    const __half *aplain;  // plain: A [n_rt * 128][K] fp16
     int direct_T;       // plain: tiles are tokens [256u, 256u + 256) of T tokens
     int out_ld;
     int *err;
@@ -87,7 +101,7 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long l
         return false;
     }
     long long t0 = clock64();
-    while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
+    while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > budget) {
             atomicCAS(err, 0, kErrTimeout);
@@ -101,24 +115,30 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long l
 __device__ __forceinline__ uint32_t h2u(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
 __device__ __forceinline__ __half2 u2h(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
 
+// silu(g) * u with the fast exponential and division (the output is rounded
+// to fp16, far coarser than their error).
+__device__ __forceinline__ float swiglu(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 template <int kBits, int kMode>
-__global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const UmmaParams p) {
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+    umma_expert_kernel(const __grid_constant__ UmmaParams p) {
     constexpr bool kGateUp = kMode == kModeGateUp;
+    constexpr bool kPlain = kMode == kModePlain;
     using Cfg = UmmaCfg<kMode>;
-    constexpr int S = Cfg::kStages, SB = Cfg::kStageBytes;
-    constexpr int UB = unit_bytes(kBits);
-    constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
-    extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *stages = smem;
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(smem + S * SB);
+    constexpr int S = Cfg::kStages, SB = Cfg::kStageBytes, NB = Cfg::kAccBufs;
+    extern __shared__ uint8_t smem_raw[];
+    // the swizzled operands need 1024-byte aligned stages
+    uint8_t *stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(stages + S * SB);
     uint64_t *full_b = full_a + S;
     uint64_t *empty = full_b + S;
-    uint64_t *acc_full = empty + S;
-    uint64_t *acc_empty = acc_full + 1;
-    uint64_t *drain = acc_empty + 1;
+    uint64_t *acc_full = empty + S;    // [NB]
+    uint64_t *acc_empty = acc_full + 2;  // [NB]
+    uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *rowoff = reinterpret_cast<int *>(tmem_slot + 4);  // [kTN] source row offsets
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -127,8 +147,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kNumEpi);
+        for (int b = 0; b < NB; b++) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kNumEpi);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -154,12 +176,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, it++) {
                 const int n = tile_unit(p, t / p.n_rt).z;
                 const uint32_t idesc = umma_idesc_f16(kTM, (n + 15) & ~15);
-                if (it > 0 && !pipe_wait(acc_empty, (it - 1) & 1, p.budget, p.err, abort_flag)) break;
+                const int buf = it % NB, use = it / NB;
+                if (use > 0 &&
+                    !pipe_wait(&acc_empty[buf], (use - 1) & 1, p.budget, p.err, abort_flag))
+                    break;
                 tc_fence_after();
+                const uint32_t dacc = tmem + buf * kTN;
                 for (int ks = 0; ks < ksteps; ks++, gs++) {
                     const int slot = gs % S;
                     const uint32_t ph = (gs / S) & 1;
-                    if (!pipe_wait(&full_a[slot], ph, p.budget, p.err, abort_flag) ||
+                    if ((!kPlain && !pipe_wait(&full_a[slot], ph, p.budget, p.err, abort_flag)) ||
                         !pipe_wait(&full_b[slot], ph, p.budget, p.err, abort_flag)) {
                         ok = false;
                         break;
@@ -169,270 +195,229 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) umma_expert_kernel(const Umma
                     const uint32_t b0 = a0 + Cfg::kMats * kTileA;
 #pragma unroll
                     for (int j = 0; j < kKS / 16; j++) {
-                        const uint64_t bd = umma_desc(b0 + j * 256, 128, 1024);
+                        const uint64_t bd = umma_desc_sw128(b0 + j * 32);
+                        const uint64_t ad = kPlain ? umma_desc_sw128(a0 + j * 32)
+                                                   : umma_desc(a0 + j * 256, 128, 1024);
                         const uint32_t acc = (ks | j) != 0;
-                        umma_f16(tmem, umma_desc(a0 + j * 256, 128, 1024), bd, idesc, acc);
+                        umma_f16(dacc, ad, bd, idesc, acc);
                         if (kGateUp)
                             umma_f16(tmem + kTN, umma_desc(a0 + kTileA + j * 256, 128, 1024), bd,
                                      idesc, acc);
                     }
                     umma_commit(&empty[slot]);
                 }
-                if (ok) umma_commit(acc_full);
+                if (ok) umma_commit(&acc_full[buf]);
             }
             // let every issued MMA finish before tensor memory is released
             umma_commit(drain);
             mbar_drain(drain, 0);
         }
-    } else if (warp == kWarpLoadB) {
-        // ---------------------------------------------------------- token rows
+    } else if (warp == kWarpLoad) {
+        // ---------------------------------------------------------- TMA loads
+        if (lane == 0) {
+            prefetch_tmap(&p.tm_b);
+            if (kPlain) prefetch_tmap(&p.tm_a);
+        }
         uint32_t gs = 0;
-        int prev = -1;
-        const int crow = lane >> 3, chunk = lane & 7;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
             const int rows = (n + 15) & ~15;
-            // the previous tile's stages only read rowoff while issuing, so it
-            // can be rewritten here (one warp, program order)
-            __syncwarp();
-            for (int r = lane; r < rows; r += 32) {
-                int off = -1;
-                if (r < n) {
-                    const int sl = slot0 + r;
-                    const int src = kGateUp ? (sl < p.Tk ? p.list[sl] : sl - p.Tk) : sl;
-                    off = src * p.K;
-                }
-                rowoff[r] = off;
-            }
-            __syncwarp();
-            bool ok = true;
+            const int rt = t % p.n_rt;
             for (int ks = 0; ks < ksteps; ks++, gs++) {
                 const int slot = gs % S;
-                if (gs >= (uint32_t)S &&
-                    !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *sB = stages + slot * SB + Cfg::kMats * kTileA;
-#pragma unroll 4
-                for (int r = crow; r < rows; r += 4) {
-                    uint8_t *dst = sB + (r >> 3) * 1024 + chunk * 128 + (r & 7) * 16;
-                    const int off = rowoff[r];
-                    const __half *src = off >= 0 ? p.xin + off + ks * kKS + chunk * 8 : p.xin;
-                    cp_async16(dst, src, off >= 0 ? 16u : 0u);
-                }
-                cp_async_commit();
-                if (prev >= 0) {
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full_b[prev]);
-                }
-                prev = slot;
-            }
-            if (!ok) break;
-        }
-        cp_async_wait<0>();
-        if (prev >= 0 && !*abort_flag) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_b[prev]);
-        }
-    } else if (kMode == kModePlain && warp < kWarpDq0 + kNumDq) {
-        // ---------------------------------------------------------- A copy
-        // 128 rows x 64 columns of fp16 per stage: 1024 16-byte chunks, each one
-        // row of one core matrix; 8 per thread, grouped per stage.
-        const int dt = threadIdx.x - 32 * kWarpDq0;
-        uint32_t gs = 0;
-        int prev = -1;
-        bool ok = true;
-        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            const int rt = t % p.n_rt;
-            const __half *abase = p.aplain + (size_t)rt * kTM * p.K;
-            for (int ks = 0; ks < ksteps; ks++, gs++) {
-                const int slot = gs % S;
-                if (gs >= (uint32_t)S &&
-                    !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *sA = stages + slot * SB;
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int idx = dt + 128 * i, r = idx >> 3, ch = idx & 7;
-                    cp_async16(sA + (r >> 3) * 1024 + ch * 128 + (r & 7) * 16,
-                               abase + (size_t)r * p.K + ks * kKS + ch * 8, 16u);
-                }
-                cp_async_commit();
-                if (prev >= 0) {
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full_a[prev]);
-                }
-                prev = slot;
-            }
-        }
-        cp_async_wait<0>();
-        if (prev >= 0 && !*abort_flag) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[prev]);
-        }
-    } else if (kMode != kModePlain && warp < kWarpDq0 + kNumDq) {
-        // ---------------------------------------------------------- dequant
-        const int dt = threadIdx.x - 32 * kWarpDq0;  // 0..127
-        const int L = dt & 31, sl0 = dt >> 5;        // slabs sl0 and sl0 + 4
-        const int g8 = L >> 2, c = L & 3;
-        const __half2 half2_05 = __float2half2_rn(0.5f);
-        // packed words of one stage for this thread: [matrix][slab]
-        struct Raw {
-            uint2 lo[Cfg::kMats][2];
-            uint32_t hi[Cfg::kMats][2];
-            uint2 sc[Cfg::kMats][2];
-        };
-        auto fetch = [&](int t, int ks, Raw &r) {
-            const int rt = t % p.n_rt;
-            const int e = __ldg(&p.units[t / p.n_rt].x);
-            const uint8_t *wbase =
-                (e == p.E ? p.shared : p.routed + (size_t)e * p.expert_bytes) + p.mat_off;
-            const int seg = ks >> 1, h = ks & 1;
-#pragma unroll
-            for (int m = 0; m < Cfg::kMats; m++)
-#pragma unroll
-                for (int si = 0; si < 2; si++) {
-                    const uint8_t *un = wbase + m * p.mat_bytes +
-                                        ((size_t)(rt * 8 + sl0 + 4 * si) * p.nseg + seg) * UB;
-                    r.lo[m][si] = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
-                    r.hi[m][si] = kBits == 3 ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                   un + kLoBytes + L * 8 + 4 * h))
-                                             : 0u;
-                    r.sc[m][si] = __ldg(
-                        reinterpret_cast<const uint2 *>(un + SOFF + (4 * g8 + 2 * h) * 4));
-                }
-        };
-        // Walk the (tile, stage) sequence with three register buffers: the raw
-        // words of position i+3 are requested right after position i is
-        // dequantised, i.e. two stages of work before they are needed.
-        struct Pos {
-            int t, ks;
-        };
-        auto advance = [&](Pos q) {
-            if (++q.ks == ksteps) {
-                q.ks = 0;
-                q.t += gridDim.x;
-            }
-            return q;
-        };
-        uint32_t gs = 0;
-        bool ok = true;
-        // returns false when the pipeline must stop (end of work or abort)
-        auto step = [&](const Raw &cur, Pos q) -> bool {
-            const int slot = gs % S;
-            if (gs >= (uint32_t)S &&
-                !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag))
-                return false;
-            const int h = q.ks & 1;
-            (void)h;
-            uint8_t *sA = stages + slot * SB;
-#pragma unroll
-            for (int m = 0; m < Cfg::kMats; m++)
-#pragma unroll
-                for (int si = 0; si < 2; si++) {
-                    const int sl = sl0 + 4 * si;
-#pragma unroll
-                    for (int bw = 0; bw < 2; bw++) {
-                        const uint32_t lw = bw ? cur.lo[m][si].y : cur.lo[m][si].x;
-                        const __half2 s2 =
-                            __hmul2(u2h(bw ? cur.sc[m][si].y : cur.sc[m][si].x), half2_05);
-                        const __half2 s_lo = __low2half2(s2), s_hi = __high2half2(s2);
-#pragma unroll
-                        for (int s = 0; s < 2; s++)
-#pragma unroll
-                            for (int r = 0; r < 4; r++) {
-                                const uint32_t pr =
-                                    kBits == 2 ? dq2_pair(lw, 4 * s + r)
-                                               : dq_pair<false, kBits>(lw, cur.hi[m][si],
-                                                                       4 * s + r, 8 * bw);
-                                const __half2 v = __hmul2(u2h(pr), (r & 1) ? s_hi : s_lo);
-                                const int R8 = 2 * sl + (r & 1);
-                                const int kc = 4 * bw + 2 * s + (r >> 1);
-                                *reinterpret_cast<uint32_t *>(sA + m * kTileA + R8 * 1024 +
-                                                              kc * 128 + g8 * 16 + 4 * c) = h2u(v);
-                            }
+                int okl = 1;
+                if (lane == 0) {
+                    if (gs >= (uint32_t)S &&
+                        !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag)) {
+                        okl = 0;
+                    } else {
+                        uint8_t *sA = stages + slot * SB;
+                        uint8_t *sB = sA + Cfg::kMats * kTileA;
+                        mbar_arrive_expect_tx(&full_b[slot],
+                                              (uint32_t)(rows * 128 + (kPlain ? kTileA : 0)));
+                        // rows past n (and past the matrix) are never read back
+                        for (int r = 0; r < rows; r += kBoxRows)
+                            tma_load_2d(sB + r * 128, &p.tm_b, ks * kKS, slot0 + r,
+                                        &full_b[slot]);
+                        if (kPlain) tma_load_2d(sA, &p.tm_a, ks * kKS, rt * kTM, &full_b[slot]);
                     }
                 }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (L == 0) mbar_arrive(&full_a[slot]);
-            gs++;
-            return true;
-        };
-        Raw r0, r1, r2;
-        Pos p0{(int)blockIdx.x, 0}, p1 = advance(p0), p2 = advance(p1);
-        if (p0.t < n_tiles) fetch(p0.t, p0.ks, r0);
-        if (p1.t < n_tiles) fetch(p1.t, p1.ks, r1);
-        if (p2.t < n_tiles) fetch(p2.t, p2.ks, r2);
-        while (ok) {
-            if (p0.t >= n_tiles || !step(r0, p0)) break;
-            const Pos p3 = advance(p2);
-            if (p3.t < n_tiles) fetch(p3.t, p3.ks, r0);
-            if (p1.t >= n_tiles || !step(r1, p1)) break;
-            const Pos p4 = advance(p3);
-            if (p4.t < n_tiles) fetch(p4.t, p4.ks, r1);
-            if (p2.t >= n_tiles || !step(r2, p2)) break;
-            const Pos p5 = advance(p4);
-            if (p5.t < n_tiles) fetch(p5.t, p5.ks, r2);
-            p0 = p3;
-            p1 = p4;
-            p2 = p5;
+                okl = __shfl_sync(0xffffffffu, okl, 0);
+                if (!okl) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        // after an abort, let the loads of the stages armed last land
+        if (lane == 0 && *abort_flag) {
+            for (uint32_t g2 = gs > (uint32_t)S ? gs - S : 0; g2 < gs; g2++)
+                mbar_drain(&full_b[g2 % S], (g2 / S) & 1);
+        }
+    } else if (warp < kWarpEpi0) {
+        if constexpr (!kPlain) {
+            // ------------------------------------------------------ dequant
+            const int dt = threadIdx.x - 32 * kWarpDq0;  // 0..127
+            const int L = dt & 31, sl0 = dt >> 5;        // slabs sl0 and sl0 + 4
+            const int g8 = L >> 2, c = L & 3;
+            constexpr int UB = unit_bytes(kBits);
+            constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
+            const __half2 half2_05 = __float2half2_rn(0.5f);
+            // packed words of one stage for this thread: [matrix][slab]
+            struct Raw {
+                uint2 lo[Cfg::kMats][2];
+                uint32_t hi[Cfg::kMats][2];
+                uint2 sc[Cfg::kMats][2];
+            };
+            auto fetch = [&](int t, int ks, Raw &r) {
+                const int rt = t % p.n_rt;
+                const int e = __ldg(&p.units[t / p.n_rt].x);
+                const uint8_t *wbase =
+                    (e == p.E ? p.shared : p.routed + (size_t)e * p.expert_bytes) + p.mat_off;
+                const int seg = ks >> 1, h = ks & 1;
+#pragma unroll
+                for (int m = 0; m < Cfg::kMats; m++)
+#pragma unroll
+                    for (int si = 0; si < 2; si++) {
+                        const uint8_t *un = wbase + m * p.mat_bytes +
+                                            ((size_t)(rt * 8 + sl0 + 4 * si) * p.nseg + seg) * UB;
+                        r.lo[m][si] = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
+                        r.hi[m][si] = kBits == 3 ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                       un + kLoBytes + L * 8 + 4 * h))
+                                                 : 0u;
+                        r.sc[m][si] = __ldg(
+                            reinterpret_cast<const uint2 *>(un + SOFF + (4 * g8 + 2 * h) * 4));
+                    }
+            };
+            // Walk the (tile, stage) sequence with three register buffers: the
+            // raw words of position i+3 are requested right after position i is
+            // dequantised, i.e. two stages of work before they are needed.
+            struct Pos {
+                int t, ks;
+            };
+            auto advance = [&](Pos q) {
+                if (++q.ks == ksteps) {
+                    q.ks = 0;
+                    q.t += gridDim.x;
+                }
+                return q;
+            };
+            uint32_t gs = 0;
+            // returns false when the pipeline must stop (abort)
+            auto step = [&](const Raw &cur) -> bool {
+                const int slot = gs % S;
+                if (gs >= (uint32_t)S &&
+                    !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag))
+                    return false;
+                uint8_t *sA = stages + slot * SB;
+#pragma unroll
+                for (int m = 0; m < Cfg::kMats; m++)
+#pragma unroll
+                    for (int si = 0; si < 2; si++) {
+                        const int sl = sl0 + 4 * si;
+#pragma unroll
+                        for (int bw = 0; bw < 2; bw++) {
+                            const uint32_t lw = bw ? cur.lo[m][si].y : cur.lo[m][si].x;
+                            const __half2 s2 =
+                                __hmul2(u2h(bw ? cur.sc[m][si].y : cur.sc[m][si].x), half2_05);
+                            const __half2 s_lo = __low2half2(s2), s_hi = __high2half2(s2);
+#pragma unroll
+                            for (int s = 0; s < 2; s++)
+#pragma unroll
+                                for (int r = 0; r < 4; r++) {
+                                    const uint32_t pr =
+                                        kBits == 2 ? dq2_pair(lw, 4 * s + r)
+                                                   : dq_pair<false, kBits>(lw, cur.hi[m][si],
+                                                                           4 * s + r, 8 * bw);
+                                    const __half2 v = __hmul2(u2h(pr), (r & 1) ? s_hi : s_lo);
+                                    const int R8 = 2 * sl + (r & 1);
+                                    const int kc = 4 * bw + 2 * s + (r >> 1);
+                                    *reinterpret_cast<uint32_t *>(sA + m * kTileA + R8 * 1024 +
+                                                                  kc * 128 + g8 * 16 + 4 * c) =
+                                        h2u(v);
+                                }
+                        }
+                    }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (L == 0) mbar_arrive(&full_a[slot]);
+                gs++;
+                return true;
+            };
+            Raw r0, r1, r2;
+            Pos p0{(int)blockIdx.x, 0}, p1 = advance(p0), p2 = advance(p1);
+            if (p0.t < n_tiles) fetch(p0.t, p0.ks, r0);
+            if (p1.t < n_tiles) fetch(p1.t, p1.ks, r1);
+            if (p2.t < n_tiles) fetch(p2.t, p2.ks, r2);
+            while (true) {
+                if (p0.t >= n_tiles || !step(r0)) break;
+                const Pos p3 = advance(p2);
+                if (p3.t < n_tiles) fetch(p3.t, p3.ks, r0);
+                if (p1.t >= n_tiles || !step(r1)) break;
+                const Pos p4 = advance(p3);
+                if (p4.t < n_tiles) fetch(p4.t, p4.ks, r1);
+                if (p2.t >= n_tiles || !step(r2)) break;
+                const Pos p5 = advance(p4);
+                if (p5.t < n_tiles) fetch(p5.t, p5.ks, r2);
+                p0 = p3;
+                p1 = p4;
+                p2 = p5;
+            }
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int q = warp & 3;  // tensor-memory lane quarter of this warp
+        const int q = warp & 3;  // tensor-memory lane quarter this warp may read
         const int r_in = 32 * q + lane;
         int it = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, it++) {
-            if (!pipe_wait(acc_full, it & 1, p.budget, p.err, abort_flag)) break;
+            const int buf = it % NB, use = it / NB;
+            if (!pipe_wait(&acc_full[buf], use & 1, p.budget, p.err, abort_flag)) break;
             tc_fence_after();
             const int rt = t % p.n_rt;
             const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
             const int row = rt * kTM + r_in;
-            for (int nc = 0; nc < kTN / 32; nc++) {
-                if (nc * 32 >= n) break;  // uniform across the warp; columns past n are ignored
+            const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + buf * kTN;
+            for (int nc = 0; nc * 32 < n; nc++) {
+                const int cnt = n - nc * 32;  // valid columns of this chunk
+                const size_t o0 = (size_t)(slot0 + nc * 32) * p.out_ld + row;
                 float gv[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + nc * 32, gv);
+                tmem_ld32(tb + nc * 32, gv);
                 if (kGateUp) {
                     float uv[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + kTN + nc * 32, uv);
+                    tmem_ld32(tb + kTN + nc * 32, uv);
+                    if (cnt >= 32) {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int tok = nc * 32 + j;
-                        if (tok < n) {
-                            const float a = gv[j] / (1.0f + __expf(-gv[j])) * uv[j];
-                            p.out[(size_t)(slot0 + tok) * p.out_ld + row] = __float2half_rn(a);
-                        }
+                        for (int j = 0; j < 32; j++)
+                            p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(swiglu(gv[j], uv[j]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (j < cnt)
+                                p.out[o0 + (size_t)j * p.out_ld] =
+                                    __float2half_rn(swiglu(gv[j], uv[j]));
                     }
                 } else if (kMode == kModeDown) {
+                    if (cnt >= 32) {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int tok = nc * 32 + j;
-                        if (tok < n)
-                            p.out[(size_t)(slot0 + tok) * p.out_ld + row] = __float2half_rn(gv[j]);
+                        for (int j = 0; j < 32; j++)
+                            p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(gv[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (j < cnt) p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(gv[j]);
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int tok = nc * 32 + j;
-                        if (tok < n) p.out32[(size_t)(slot0 + tok) * p.out_ld + row] = gv[j];
-                    }
+                    for (int j = 0; j < 32; j++)
+                        if (j < cnt) p.out32[o0 + (size_t)j * p.out_ld] = gv[j];
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
     tc_fence_before();
@@ -455,18 +440,72 @@ __global__ void to_half_kernel(const __nv_bfloat16 *__restrict__ x, __half *__re
     reinterpret_cast<uint4 *>(y)[i] = o;
 }
 
+// ------------------------------------------------------------------- host
 static int g_num_sms = 0;
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links the runtime statically and not the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Tensor map of an fp16 matrix [rows][cols] (row pitch cols), boxes of 64
+// columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+// base 16-byte aligned and cols a multiple of 8 (the map's own checks).
+static cudaError_t encode_fp16_map(CUtensorMap *m, const void *base, int cols, int rows,
+                                   int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kKS, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims,
+                    strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int kBits, int kMode>
-static void run_umma(const UmmaParams &p, int max_tiles, cudaStream_t s) {
+static cudaError_t run_umma(const UmmaParams &p, int max_tiles, cudaStream_t s) {
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     int grid = max_tiles < g_num_sms ? max_tiles : g_num_sms;
-    if (grid <= 0) return;
+    if (grid <= 0) return cudaSuccess;
     umma_expert_kernel<kBits, kMode><<<grid, kUmmaThreads, UmmaCfg<kMode>::kSmem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// xs[slot] = x16[list[slot]] for the Tk routed slots (one warp per row,
+// 16-byte copies); the shared expert's rows follow as x16 itself.
+__global__ void gather_rows_kernel(const int32_t *__restrict__ list, int Tk,
+                                   const uint4 *__restrict__ x16, uint4 *__restrict__ xs,
+                                   int row16) {
+    const int slot = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (slot >= Tk) return;
+    const uint4 *src = x16 + (size_t)__ldg(list + slot) * row16;
+    uint4 *dst = xs + (size_t)slot * row16;
+    for (int i = lane; i < row16; i += 32) dst[i] = __ldg(src + i);
+}
+
+void launch_gather_rows(const int32_t *list, int Tk, const void *x16, void *xs, int H,
+                        cudaStream_t s) {
+    if (Tk <= 0) return;
+    gather_rows_kernel<<<(unsigned)((Tk + 7) / 8), 256, 0, s>>>(
+        list, Tk, reinterpret_cast<const uint4 *>(x16), reinterpret_cast<uint4 *>(xs), H / 8);
 }
 
 void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s) {
@@ -493,47 +532,46 @@ static UmmaParams base_params(const Geometry &g, const ExpertWeights &w, const i
     return p;
 }
 
-void launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                        const int *n_units, int units_max, const int32_t *list, int Tk,
-                        const void *x16, void *a, int *err, long long budget, cudaStream_t s) {
-    // A = Wg, Wu (Ip rows, K = H); B = x rows (fp16 copy) gathered by token
-    UmmaParams p = base_params(g, w, units, n_units, list, Tk, err, budget);
+cudaError_t launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                               const int *n_units, int units_max, int slots, const void *xs,
+                               void *a, int *err, long long budget, cudaStream_t s) {
+    // A = Wg, Wu (Ip rows, K = H); B = token rows by slot
+    UmmaParams p = base_params(g, w, units, n_units, nullptr, 0, err, budget);
+    cudaError_t e = encode_fp16_map(&p.tm_b, xs, g.H, slots, kBoxRows);
+    if (e != cudaSuccess) return e;
     p.mat_off = 0;
-    p.xin = reinterpret_cast<const __half *>(x16);
     p.K = g.H;
     p.nseg = g.H / kSegCols;
     p.n_rt = g.Ip / kTM;
     p.out = reinterpret_cast<__half *>(a);
     p.out_ld = g.Ip;
-    if (g.bits == 2)
-        run_umma<2, kModeGateUp>(p, units_max * p.n_rt, s);
-    else
-        run_umma<3, kModeGateUp>(p, units_max * p.n_rt, s);
+    return g.bits == 2 ? run_umma<2, kModeGateUp>(p, units_max * p.n_rt, s)
+                       : run_umma<3, kModeGateUp>(p, units_max * p.n_rt, s);
 }
 
-void launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
-                      const int *n_units, int units_max, const void *a, void *Y, int *err,
-                      long long budget, cudaStream_t s) {
+cudaError_t launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
+                             const int *n_units, int units_max, int slots, const void *a, void *Y,
+                             int *err, long long budget, cudaStream_t s) {
     // A = Wd (H rows, K = Ip); B = a rows by slot
     UmmaParams p = base_params(g, w, units, n_units, nullptr, 0, err, budget);
+    cudaError_t e = encode_fp16_map(&p.tm_b, a, g.Ip, slots, kBoxRows);
+    if (e != cudaSuccess) return e;
     p.mat_off = 2 * g.mat_bytes;
-    p.xin = reinterpret_cast<const __half *>(a);
     p.K = g.Ip;
     p.nseg = g.Ip / kSegCols;
     p.n_rt = g.H / kTM;
     p.out = reinterpret_cast<__half *>(Y);
     p.out_ld = g.H;
-    if (g.bits == 2)
-        run_umma<2, kModeDown>(p, units_max * p.n_rt, s);
-    else
-        run_umma<3, kModeDown>(p, units_max * p.n_rt, s);
+    return g.bits == 2 ? run_umma<2, kModeDown>(p, units_max * p.n_rt, s)
+                       : run_umma<3, kModeDown>(p, units_max * p.n_rt, s);
 }
 
-void launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
-                       int *err, long long budget, cudaStream_t s) {
+cudaError_t launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
+                              int *err, long long budget, cudaStream_t s) {
     UmmaParams p{};
-    p.aplain = A;
-    p.xin = x16;
+    cudaError_t e = encode_fp16_map(&p.tm_b, x16, K, T, kBoxRows);
+    if (e == cudaSuccess) e = encode_fp16_map(&p.tm_a, A, K, rows, kTM);
+    if (e != cudaSuccess) return e;
     p.direct_T = T;
     p.K = K;
     p.nseg = K / kSegCols;
@@ -542,10 +580,12 @@ void launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int 
     p.out_ld = rows;
     p.err = err;
     p.budget = budget;
-    run_umma<2, kModePlain>(p, ((T + kTN - 1) / kTN) * p.n_rt, s);
+    return run_umma<2, kModePlain>(p, ((T + kTN - 1) / kTN) * p.n_rt, s);
 }
 
 cudaError_t umma_init_attributes(int max_smem) {
+    // look the encoder up here, outside any stream capture
+    if (!encode_fn()) return cudaErrorNotSupported;
     cudaError_t e;
     if ((e = allow_max_dyn_smem(umma_expert_kernel<2, kModeGateUp>, max_smem)) != cudaSuccess)
         return e;

@@ -253,3 +253,68 @@ def test_screened_router_ties_and_near_ties(T):
     zero.router_w = np.zeros_like(base.router_w)
     zero.router_b = np.zeros_like(base.router_b)
     _route_case(zero, T, 7, "zero router")
+
+
+def _tie_layers(shape, seed):
+    """The layer plus three router variants: duplicated rows (exact ties, the
+    lower id wins), rows one ulp apart, and an all-zero router (every logit
+    ties)."""
+    import copy
+    base = gen.layer_weights(shape, seed=seed)
+    out = [("base", base)]
+    dup = copy.copy(base)
+    W = base.router_w.copy()
+    W[1::2] = W[0::2]
+    b = base.router_b.copy() if base.router_b is not None else None
+    if b is not None:
+        b[1::2] = b[0::2]
+    dup.router_w, dup.router_b = W, b
+    out.append(("duplicated rows", dup))
+    near = copy.copy(base)
+    W2 = base.router_w.copy()
+    W2[1::2] = np.nextafter(W2[0::2], np.float32(np.inf))
+    near.router_w, near.router_b = W2, b
+    out.append(("one-ulp rows", near))
+    zero = copy.copy(base)
+    zero.router_w = np.zeros_like(base.router_w)
+    zero.router_b = None if base.router_b is None else np.zeros_like(base.router_b)
+    out.append(("zero router", zero))
+    return out
+
+
+@pytest.mark.parametrize("T", [1, 4, 13, 64])
+def test_fused_decode_equals_gemv_chain(T):
+    """The fused decode kernel (router top-k in the router's last CTA, dispatch,
+    gate/up, down and combine in one launch) does the same arithmetic in the
+    same order as the chain of decode kernels, so the two outputs are equal bit
+    for bit, also where the routing meets exact ties and one-ulp near-ties;
+    and both match the oracle."""
+    shape = gen.LayerShape(hidden=512, n_experts=512, top_k=10, inter=128, bits=2,
+                           router_bias=True)
+    for label, w in _tie_layers(shape, seed=41):
+        x = gen.hidden(T, shape.hidden, seed=42)
+        xt = to_dev_bf16(x)
+        fused = qe.Layer(w, max_tokens=T)
+        fused.set_option(qe.STRATA_OPT_PATH, 3)
+        chain = qe.Layer(w, max_tokens=T)
+        chain.set_option(qe.STRATA_OPT_PATH, 1)
+        assert qe.strata_moe_launch_count(fused.handle, T) == 2
+        yf = from_dev_bf16(fused.forward(xt))
+        yc = from_dev_bf16(chain.forward(xt))
+        fused.sync_status()
+        chain.sync_status()
+        assert np.array_equal(yf, yc), f"T={T} {label}: fused and chained outputs differ"
+        _, ref, _, _ = oracle.moe_forward(w, x, threads=THREADS)
+        check_output(yf, ref, f"fused T={T} {label}")
+
+
+def test_fused_decode_3bit_batch():
+    """3-bit weights at the batched-decode size, fused against the chain."""
+    shape, T = gen.FLASH3, 64
+    x = to_dev_bf16(gen.hidden(T, shape.hidden, seed=43))
+    fused = gpu_layer(shape, T, path=3)
+    chain = gpu_layer(shape, T, path=1)
+    yf = from_dev_bf16(fused.forward(x))
+    yc = from_dev_bf16(chain.forward(x))
+    fused.sync_status()
+    assert np.array_equal(yf, yc)
