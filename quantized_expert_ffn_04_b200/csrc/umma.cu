@@ -11,7 +11,7 @@
 // the tile's token count rounded up to 16, so a cold expert's short tile does
 // not pay for empty columns), K in stages of 64.  Operands are fp16, K-major.
 // The token operand B is brought in by the tensor memory accelerator with the
-// 128-byte swizzle, 16 consecutive rows per box: gate/up reads the fp16 token
+// 128-byte swizzle, 64 consecutive rows per box: gate/up reads the fp16 token
 // rows in slot order (each expert's tokens contiguous, built once per forward
 // by gather_rows_kernel), down reads a by slot, the plain GEMM reads x.  The weight
 // operand A is written by the dequant warps without swizzle, in 8-row x
@@ -19,7 +19,7 @@
 // 1024 B apart); the plain GEMM loads A by tensor map as well.  Warp roles:
 //   warp 0      allocates tensor memory; lane 0 issues the MMAs and commits
 //               them to the stage and accumulator barriers;
-//   warp 1      lane 0 issues the tensor-map loads of each stage;
+//   warp 1      issues the tensor-map loads of each stage, one box per lane;
 //   warps 2..5  dequantise the weight tile into the A operand: codes -> exact
 //               odd integers -> one packed multiply by d/2, i.e. the fp16 value
 //               of d*(q-c) rounded once to nearest even;
@@ -45,7 +45,7 @@ constexpr int kTN = 256;                // most tokens per tile
 constexpr int kKS = 64;                 // K per stage (one 128-byte swizzle row)
 constexpr int kTileA = kTM * kKS * 2;   // 16 KB
 constexpr int kTileB = kTN * kKS * 2;   // 32 KB
-constexpr int kBoxRows = 16;            // rows per 2-D box of the token operand
+constexpr int kBoxRows = 64;            // rows per 2-D box of the token operand (8 KB)
 constexpr int kWarpMma = 0, kWarpLoad = 1, kWarpDq0 = 2, kNumDq = 4, kWarpEpi0 = 6, kNumEpi = 4;
 constexpr int kUmmaThreads = 32 * 10;
 
@@ -54,15 +54,21 @@ constexpr int kUmmaThreads = 32 * 10;
 // tensor map, fp32 out; used by the router's screening GEMM).
 constexpr int kModeGateUp = 0, kModeDown = 1, kModePlain = 2;
 
+// Separate rings for the two operands: the dequantised weight tile (A) is
+// made on the SM (three slots let the dequant run two stages ahead of the
+// MMAs), while the token rows (B) arrive from L2/HBM with microseconds of
+// latency and get the rest of shared memory.
+// The plain GEMM loads A by tensor map as well, in the same number of slots.
 template <int kMode>
 struct UmmaCfg {
     static constexpr int kMats = kMode == kModeGateUp ? 2 : 1;
-    static constexpr int kStages = kMode == kModeGateUp ? 3 : 4;
-    static constexpr int kStageBytes = kMats * kTileA + kTileB;
+    static constexpr int kStagesB = kMode == kModeGateUp ? 4 : (kMode == kModeDown ? 5 : 4);
+    static constexpr int kStagesA = kMode == kModePlain ? kStagesB : 3;
+    static constexpr int kSlotA = kMats * kTileA;
     static constexpr int kAccBufs = kMode == kModeGateUp ? 1 : 2;
     static constexpr int kTmemCols = 512;
-    // stages + alignment slack (1024) + barriers
-    static constexpr int kSmem = kStages * kStageBytes + 1024 + 2048;
+    // A ring + B ring + alignment slack (1024) + barriers
+    static constexpr int kSmem = kStagesA * kSlotA + kStagesB * kTileB + 1024 + 2048;
 };
 
 struct UmmaParams {
@@ -95,6 +101,8 @@ __device__ __forceinline__ int4 tile_unit(const UmmaParams &p, int u) {
 
 __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long long budget,
                                           int *err, volatile int *abort_flag) {
+    // fast path: the phase is usually complete already
+    if (mbar_test_wait(bar, parity)) return true;
     if (budget <= 0) {
         atomicCAS(err, 0, kErrTimeout);
         *abort_flag = 1;
@@ -127,14 +135,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     constexpr bool kGateUp = kMode == kModeGateUp;
     constexpr bool kPlain = kMode == kModePlain;
     using Cfg = UmmaCfg<kMode>;
-    constexpr int S = Cfg::kStages, SB = Cfg::kStageBytes, NB = Cfg::kAccBufs;
+    constexpr int SA = Cfg::kStagesA, SBn = Cfg::kStagesB, NB = Cfg::kAccBufs;
     extern __shared__ uint8_t smem_raw[];
-    // the swizzled operands need 1024-byte aligned stages
-    uint8_t *stages = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(stages + S * SB);
-    uint64_t *full_b = full_a + S;
-    uint64_t *empty = full_b + S;
-    uint64_t *acc_full = empty + S;    // [NB]
+    // the swizzled operands need 1024-byte aligned slots
+    uint8_t *ringA = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *ringB = ringA + SA * Cfg::kSlotA;
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(ringB + SBn * kTileB);
+    uint64_t *empty_a = full_a + SA;
+    uint64_t *full_b = empty_a + SA;
+    uint64_t *empty_b = full_b + SBn;
+    uint64_t *acc_full = empty_b + SBn;  // [NB]
     uint64_t *acc_empty = acc_full + 2;  // [NB]
     uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -142,10 +152,13 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; s++) {
+        for (int s = 0; s < SA; s++) {
             mbar_init(&full_a[s], kNumDq);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < SBn; s++) {
             mbar_init(&full_b[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty_b[s], 1);
         }
         for (int b = 0; b < NB; b++) {
             mbar_init(&acc_full[b], 1);
@@ -183,28 +196,30 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                 tc_fence_after();
                 const uint32_t dacc = tmem + buf * kTN;
                 for (int ks = 0; ks < ksteps; ks++, gs++) {
-                    const int slot = gs % S;
-                    const uint32_t ph = (gs / S) & 1;
-                    if ((!kPlain && !pipe_wait(&full_a[slot], ph, p.budget, p.err, abort_flag)) ||
-                        !pipe_wait(&full_b[slot], ph, p.budget, p.err, abort_flag)) {
+                    const int sa = gs % SA, sb = gs % SBn;
+                    if ((!kPlain && !pipe_wait(&full_a[sa], (gs / SA) & 1, p.budget, p.err,
+                                               abort_flag)) ||
+                        !pipe_wait(&full_b[sb], (gs / SBn) & 1, p.budget, p.err, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(stages + slot * SB);
-                    const uint32_t b0 = a0 + Cfg::kMats * kTileA;
+                    // descriptors: the start address sits in the low bits (16-byte
+                    // units), so the K steps inside a stage are plain additions
+                    const uint64_t bd0 = umma_desc_sw128(smem_u32(ringB + sb * kTileB));
+                    const uint32_t a0 = smem_u32(ringA + sa * Cfg::kSlotA);
+                    const uint64_t ad0 = kPlain ? umma_desc_sw128(a0) : umma_desc(a0, 128, 1024);
 #pragma unroll
                     for (int j = 0; j < kKS / 16; j++) {
-                        const uint64_t bd = umma_desc_sw128(b0 + j * 32);
-                        const uint64_t ad = kPlain ? umma_desc_sw128(a0 + j * 32)
-                                                   : umma_desc(a0 + j * 256, 128, 1024);
+                        const uint64_t bd = bd0 + (uint64_t)(j * 32 >> 4);
+                        const uint64_t ad = ad0 + (uint64_t)((kPlain ? j * 32 : j * 256) >> 4);
                         const uint32_t acc = (ks | j) != 0;
                         umma_f16(dacc, ad, bd, idesc, acc);
                         if (kGateUp)
-                            umma_f16(tmem + kTN, umma_desc(a0 + kTileA + j * 256, 128, 1024), bd,
-                                     idesc, acc);
+                            umma_f16(tmem + kTN, ad + (uint64_t)(kTileA >> 4), bd, idesc, acc);
                     }
-                    umma_commit(&empty[slot]);
+                    umma_commit(&empty_b[sb]);
+                    if (!kPlain) umma_commit(&empty_a[sa]);
                 }
                 if (ok) umma_commit(&acc_full[buf]);
             }
@@ -223,38 +238,41 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
-            const int rows = (n + 15) & ~15;
+            // whole 64-row boxes (each issue costs about as much as a box's
+            // bytes take to land, so few large boxes); rows past n are never
+            // read back
+            const int nbox = (n + kBoxRows - 1) / kBoxRows;
             const int rt = t % p.n_rt;
             for (int ks = 0; ks < ksteps; ks++, gs++) {
-                const int slot = gs % S;
+                const int slot = gs % SBn;
                 int okl = 1;
                 if (lane == 0) {
-                    if (gs >= (uint32_t)S &&
-                        !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag)) {
+                    if (gs >= (uint32_t)SBn && !pipe_wait(&empty_b[slot], ((gs / SBn) + 1) & 1,
+                                                          p.budget, p.err, abort_flag))
                         okl = 0;
-                    } else {
-                        uint8_t *sA = stages + slot * SB;
-                        uint8_t *sB = sA + Cfg::kMats * kTileA;
-                        mbar_arrive_expect_tx(&full_b[slot],
-                                              (uint32_t)(rows * 128 + (kPlain ? kTileA : 0)));
-                        // rows past n (and past the matrix) are never read back
-                        for (int r = 0; r < rows; r += kBoxRows)
-                            tma_load_2d(sB + r * 128, &p.tm_b, ks * kKS, slot0 + r,
-                                        &full_b[slot]);
-                        if (kPlain) tma_load_2d(sA, &p.tm_a, ks * kKS, rt * kTM, &full_b[slot]);
-                    }
+                    else
+                        mbar_arrive_expect_tx(&full_b[slot], (uint32_t)(nbox * kBoxRows * 128 +
+                                                                        (kPlain ? kTileA : 0)));
                 }
                 okl = __shfl_sync(0xffffffffu, okl, 0);
                 if (!okl) {
                     ok = false;
                     break;
                 }
+                // the stage's boxes go out from several lanes at once
+                uint8_t *sA = ringA + (gs % SA) * Cfg::kSlotA;  // plain: SA == SBn
+                uint8_t *sB = ringB + slot * kTileB;
+                if (lane < nbox)
+                    tma_load_2d(sB + lane * kBoxRows * 128, &p.tm_b, ks * kKS,
+                                slot0 + lane * kBoxRows, &full_b[slot]);
+                if (kPlain && lane == nbox)
+                    tma_load_2d(sA, &p.tm_a, ks * kKS, rt * kTM, &full_b[slot]);
             }
         }
         // after an abort, let the loads of the stages armed last land
         if (lane == 0 && *abort_flag) {
-            for (uint32_t g2 = gs > (uint32_t)S ? gs - S : 0; g2 < gs; g2++)
-                mbar_drain(&full_b[g2 % S], (g2 / S) & 1);
+            for (uint32_t g2 = gs > (uint32_t)SBn ? gs - SBn : 0; g2 < gs; g2++)
+                mbar_drain(&full_b[g2 % SBn], (g2 / SBn) & 1);
         }
     } else if (warp < kWarpEpi0) {
         if constexpr (!kPlain) {
@@ -307,11 +325,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             uint32_t gs = 0;
             // returns false when the pipeline must stop (abort)
             auto step = [&](const Raw &cur) -> bool {
-                const int slot = gs % S;
-                if (gs >= (uint32_t)S &&
-                    !pipe_wait(&empty[slot], ((gs / S) + 1) & 1, p.budget, p.err, abort_flag))
+                const int slot = gs % SA;
+                if (gs >= (uint32_t)SA &&
+                    !pipe_wait(&empty_a[slot], ((gs / SA) + 1) & 1, p.budget, p.err, abort_flag))
                     return false;
-                uint8_t *sA = stages + slot * SB;
+                uint8_t *sA = ringA + slot * Cfg::kSlotA;
 #pragma unroll
                 for (int m = 0; m < Cfg::kMats; m++)
 #pragma unroll
