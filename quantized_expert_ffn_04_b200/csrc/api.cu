@@ -85,7 +85,7 @@ struct strata_moe {
     // routed token rows in slot order, then (at row T * k) the fp16 copy of x
     void *xs = nullptr;
     float *dsplit = nullptr;  // [max_tokens][router_rows] screening GEMM output (T > 256)
-    // fused decode counters: [units (tile 8)] then [max_tokens][H / 128]
+    // fused decode counters: [units (tile 8)], [max_tokens][H / 128], item queues [2]
     int *fused_cnt = nullptr;
     int *tok_groups = nullptr;  // router top-k counters (one per token group, self-resetting)
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
@@ -170,7 +170,7 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->xn = take(T * H * 2);
     h->xs = take(slots * H * 2);
     h->dsplit = (float *)take(T > (size_t)kSmallMaxT ? T * (size_t)h->router_rows * 4 : 0);
-    h->fused_cnt = (int *)take(((size_t)units + T * (H / 128)) * 4);
+    h->fused_cnt = (int *)take(((size_t)units + T * (H / 128) + 2) * 4);
     h->tok_groups = (int *)take(64 * 4);
     return off;
 }
@@ -280,13 +280,15 @@ strata_status run_forward_fused(strata_moe_t h, const void *x, int T, void *y, b
     const int umax = max_units(T, g.k, g.E, 8);
     probe(h, kStRouter, true, s);
     launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s, x16_of(h, T),
-                  h->fused_cnt, umax + T * (g.H / 128), g.k, h->idx, h->wts, h->tok_groups);
+                  h->fused_cnt, umax + T * (g.H / 128) + 2, g.k, h->idx, h->wts, h->tok_groups);
     probe(h, kStRouter, false, s);
     ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
     probe(h, kStGateUp, true, s);
     cudaError_t ce = launch_fused_decode(g, w, h->idx, h->wts, x16_of(h, T), T, umax, h->a,
                                          (float *)h->Y, y, residual, h->fused_cnt,
-                                         h->fused_cnt + umax, h->err, h->budget, s);
+                                         h->fused_cnt + umax,
+                                         h->fused_cnt + umax + T * (g.H / 128), h->err,
+                                         h->budget, s);
     probe(h, kStGateUp, false, s);
     if (ce != cudaSuccess)
         return fail(STRATA_ERR_CUDA, "fused decode kernel: %s", cudaGetErrorString(ce));

@@ -62,6 +62,7 @@ struct FusedParams {
     int residual;
     int *done_gu;          // [units_max] finished gate/up slabs per unit
     int *done_tok;         // [T][H / 128] finished down items per (token, row block)
+    int *queue;            // [2] next gate/up item, next down item (claimed by CTAs)
     int *err;
     long long budget;
 };
@@ -89,7 +90,7 @@ __host__ __device__ inline FusedSmem fused_smem(int T, int E, int k, int H, int 
     s.soff = o;  o += align16(E * 4);
     s.units = o; o += units_max * 16;
     s.slist = o; o += align16(T * k * 4);
-    s.misc = o;  o += 512;                       // flags, scan scratch, combine lists
+    s.misc = o;  o += 512;                       // flags, scan scratch, combine lists, item ids
     s.bars = o;  o += 8 * (2 * kFMaxRing + 2 + kFGroups);
     s.total = o;
     return s;
@@ -233,9 +234,12 @@ STRATA_DEV void group_sync(int group) {
     asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory");
 }
 
-// misc ints: [1] abort flag, [2..34] scan scratch, [36 + g] group go/stop
-// flags, [40 + 9 g] combine list of group g (count, then up to 8 tokens)
-constexpr int kMiscAbort = 1, kMiscScan = 2, kMiscFlag = 36, kMiscComb = 40;
+// misc ints: [1] abort flag, [2..34] scan scratch, [36 + g] and [88 + g]
+// group go/stop flags, [40 + 9 g] combine list of group g (count, then up to
+// 8 tokens), [80 + slot] item id of each ring slot
+constexpr int kMiscAbort = 1, kMiscScan = 2, kMiscFlag = 36, kMiscComb = 40, kMiscMeta = 80,
+              kMiscFlag2 = 88;
+constexpr int kItemEnd = -1;  // ring slot marker: no more items for this CTA
 
 template <int kBits>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedParams p) {
@@ -321,11 +325,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     const int nsl = p.Ip / kSlabRows;                 // gate/up items per unit
     const int ndn = H / (kSlabRows * kDownSlabs);     // down items per unit
     const int N1 = n_units * nsl, N2 = n_units * ndn;
-    const int G = gridDim.x, c = blockIdx.x;
-    const int g0 = (int)((long long)c * N1 / G), g1 = (int)((long long)(c + 1) * N1 / G);
-    const int d0 = (int)((long long)c * N2 / G), d1 = (int)((long long)(c + 1) * N2 / G);
-    const int len1 = g1 - g0, Lc = len1 + (d1 - d0);
-    const bool staged = p.staged && len1 > 0;
+    // items are claimed from two global queues (gate/up first, then down):
+    // a CTA that finishes early takes more, so the last CTA does not trail
+    const bool staged = p.staged != 0;
+    int *meta = misc + kMiscMeta;  // item id of each ring slot (or kItemEnd)
     const size_t gu_bytes = (size_t)p.nseg_h * UB, dn_bytes = (size_t)kDownSlabs * p.nseg_i * UB;
 
     if (warp == kFWarps) {
@@ -337,14 +340,32 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                     bulk_g2s(xs + (size_t)t * (H + 8), p.x16 + (size_t)t * H, (uint32_t)(H * 2),
                              xbar);
             }
-            int j = 0;
-            for (; j < Lc; j++) {
+            // claim items until both queues are empty, then leave one end
+            // marker per group (a marker completes its slot with no bytes)
+            int j = 0, ended = 0;
+            bool gu_left = true, dn_left = true;
+            for (; ended < kFGroups; j++) {
                 const int slot = j % p.ring;
                 if (j >= p.ring && !fwait(&empty[slot], ((j / p.ring) - 1) & 1, p, abort_flag))
                     break;
+                int item = kItemEnd;
+                if (gu_left) {
+                    const int gq = atomicAdd(p.queue, 1);
+                    if (gq < N1) item = gq;
+                    else gu_left = false;
+                }
+                if (item == kItemEnd && dn_left) {
+                    const int dq = atomicAdd(p.queue + 1, 1);
+                    if (dq < N2) item = N1 + dq;
+                    else dn_left = false;
+                }
+                meta[slot] = item;  // published by the arrive below
                 uint8_t *dst = ring + (size_t)slot * p.item_bytes;
-                if (j < len1) {
-                    const int gi = g0 + j, u = gi / nsl, slab = gi % nsl;
+                if (item == kItemEnd) {
+                    mbar_arrive(&full[slot]);
+                    ended++;
+                } else if (item < N1) {
+                    const int u = item / nsl, slab = item % nsl;
                     const int e = units[u].x;
                     const uint8_t *wg = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
                                         (size_t)slab * gu_bytes;
@@ -352,7 +373,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                     bulk_g2s(dst, wg, (uint32_t)gu_bytes, &full[slot]);
                     bulk_g2s(dst + gu_bytes, wg + p.mat_bytes, (uint32_t)gu_bytes, &full[slot]);
                 } else {
-                    const int di = d0 + (j - len1), u = di / ndn, rg = di % ndn;
+                    const int di = item - N1, u = di / ndn, rg = di % ndn;
                     const int e = units[u].x;
                     const uint8_t *wd = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
                                         2 * p.mat_bytes + (size_t)rg * dn_bytes;
@@ -374,6 +395,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     const int g = lane >> 2, cq = lane & 3;
     const int per_blk = k + 1;  // down items that write one (token, row block)
     int *flag = misc + kMiscFlag + gi;
+    int *flag2 = misc + kMiscFlag2 + gi;  // second go/stop word of a down item
     int *comb = misc + kMiscComb + 9 * gi;
     __half *abuf = reinterpret_cast<__half *>(sm + L.abuf) + (size_t)gi * kFTile * (p.Ip + 8);
     uint32_t a_uses = 0;  // phases of abar[gi] used so far (thread gtid 0)
@@ -384,27 +406,23 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
         if (!*flag) return;
         group_sync(gi);
     }
-    for (int j = gi; j < Lc; j += kFGroups) {
+    for (int j = gi;; j += kFGroups) {
         const int slot = j % p.ring;
-        const bool is_gu = j < len1;
-        int u, part;
-        if (is_gu) {
-            const int gidx = g0 + j;
-            u = gidx / nsl;
-            part = gidx % nsl;
-        } else {
-            const int di = d0 + (j - len1);
-            u = di / ndn;
-            part = di % ndn;
-        }
+        if (gtid == 0) *flag = fwait(&full[slot], (j / p.ring) & 1, p, abort_flag) ? 1 : 0;
+        group_sync(gi);
+        if (!*flag) return;  // the whole group leaves together
+        const int item = meta[slot];
+        if (item == kItemEnd) break;
+        const bool is_gu = item < N1;
+        const int u = is_gu ? item / nsl : (item - N1) / ndn;
+        const int part = is_gu ? item % nsl : (item - N1) % ndn;
         const int4 un = units[u];
         const int slot0 = un.y, n = un.z;
-        if (gtid == 0) {
-            bool ok = fwait(&full[slot], (j / p.ring) & 1, p, abort_flag);
+        if (!is_gu) {
             // a down item needs every gate/up slab of its unit (other CTAs);
             // then its n activation rows come in with one bulk copy each
-            if (ok && !is_gu) {
-                ok = fwait_count(p.done_gu + u, nsl, p, abort_flag);
+            if (gtid == 0) {
+                bool ok = fwait_count(p.done_gu + u, nsl, p, abort_flag);
                 if (ok) {
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     mbar_arrive_expect_tx(&abar[gi], (uint32_t)(n * p.Ip * 2));
@@ -415,11 +433,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                     if (!ok) mbar_drain(&abar[gi], a_uses & 1);
                     a_uses++;
                 }
+                *flag2 = ok ? 1 : 0;
             }
-            *flag = ok ? 1 : 0;
+            group_sync(gi);
+            if (!*flag2) return;
         }
-        group_sync(gi);
-        if (!*flag) return;  // the whole group leaves together
         const uint8_t *w = ring + (size_t)slot * p.item_bytes;
         if (is_gu) {
             // ------------------------------------------------ gate/up item
@@ -534,8 +552,8 @@ size_t fused_item_bytes(const Geometry &g) {
 cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const int32_t *idx,
                                 const float *wts, const void *x16, int T, int units_max, void *a,
                                 float *Y,
-                                void *out, bool residual, int *done_gu, int *done_tok, int *err,
-                                long long budget, cudaStream_t s) {
+                                void *out, bool residual, int *done_gu, int *done_tok, int *queue,
+                                int *err, long long budget, cudaStream_t s) {
     if (!fused_decode_supported(g, T) || g_fused_max_smem == 0) return cudaErrorInvalidValue;
     FusedParams p{};
     p.routed = w.routed;
@@ -560,6 +578,7 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     p.residual = residual ? 1 : 0;
     p.done_gu = done_gu;
     p.done_tok = done_tok;
+    p.queue = queue;
     p.err = err;
     p.budget = budget;
     // ring depth and token staging from the shared memory left over

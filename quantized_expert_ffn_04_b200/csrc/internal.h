@@ -109,13 +109,13 @@ cudaError_t umma_init_attributes(int max_smem);
 // After launch_router(..., x16, counters, units_max + T (H / 128), k, idx, w,
 // tok_done): dispatch, gate/up, down and combine in one kernel (programmatic
 // dependent launch).
-// done_gu [units_max] and done_tok [T][H / 128] are the router-zeroed counters.
+// done_gu [units_max], done_tok [T][H / 128] and queue [2] are router-zeroed counters.
 int fused_decode_supported(const Geometry &g, int T);
 cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const int32_t *idx,
                                 const float *wts, const void *x16, int T, int units_max, void *a,
                                 float *Y,
-                                void *out, bool residual, int *done_gu, int *done_tok, int *err,
-                                long long budget, cudaStream_t s);
+                                void *out, bool residual, int *done_gu, int *done_tok, int *queue,
+                                int *err, long long budget, cudaStream_t s);
 cudaError_t fused_init_attributes(int max_smem);
 
 // ---- combine.cu
