@@ -80,6 +80,7 @@ struct strata_moe {
     void *a = nullptr;            // fp16 [slots][Ip]
     void *Y = nullptr;            // fp32 (decode) / fp16 (prefill) [slots][H]
     int *err = nullptr;
+    int *err_host = nullptr;  // pinned copy of the error word (one sync per host forward)
     void *xio = nullptr, *yio = nullptr, *xn = nullptr;  // bf16 [max_tokens][H]
     // fp16 token operand of the tensor-core path, [max_tokens * k + max_tokens][H]:
     // routed token rows in slot order, then (at row T * k) the fp16 copy of x
@@ -182,6 +183,7 @@ void free_handle(strata_moe *h) {
     cudaFree(h->router_b);
     cudaFree(h->router_split);
     cudaFree(h->ws);
+    if (h->err_host) cudaFreeHost(h->err_host);
     delete h;
 }
 
@@ -410,6 +412,12 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
     }
     h->ws_bytes = ws_bytes;
     carve_workspace(h, (char *)h->ws);
+    if ((ce = cudaMallocHost(&h->err_host, 4)) != cudaSuccess) {
+        h->err_host = nullptr;
+        free_handle(h);
+        return cuda_fail(ce, "cudaMallocHost(error word)");
+    }
+    *h->err_host = 0;
     if ((ce = cudaMemset(h->ws, 0, ws_bytes)) != cudaSuccess) {
         free_handle(h);
         return cuda_fail(ce, "cudaMemset(workspace)");
@@ -583,14 +591,17 @@ strata_status strata_moe_sync_status(strata_moe_t h, void *stream) {
     if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
     DeviceGuard guard(h->device);
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t ce = cudaStreamSynchronize(s);
-    if (ce != cudaSuccess) return cuda_fail(ce, "stream synchronize");
-    int e = 0;
-    ce = cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost);
+    // the error word rides on the stream after the work it reports on, so one
+    // synchronisation covers both
+    cudaError_t ce = cudaMemcpyAsync(h->err_host, h->err, 4, cudaMemcpyDeviceToHost, s);
     if (ce != cudaSuccess) return cuda_fail(ce, "error word read");
+    ce = cudaStreamSynchronize(s);
+    if (ce != cudaSuccess) return cuda_fail(ce, "stream synchronize");
+    const int e = *h->err_host;
     if (e) {
-        int z = 0;
-        cudaMemcpy(h->err, &z, 4, cudaMemcpyHostToDevice);
+        *h->err_host = 0;
+        cudaMemsetAsync(h->err, 0, 4, s);
+        cudaStreamSynchronize(s);
         return fail(STRATA_ERR_TIMEOUT, "a device-side wait gave up (code %d)", e);
     }
     return STRATA_OK;

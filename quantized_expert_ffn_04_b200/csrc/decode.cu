@@ -475,9 +475,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                     const int row = part * kSlabRows + g + 8 * (i >> 1);
                     if (tok < n) p.a[(size_t)(slot0 + tok) * p.Ip + row] = __float2half_rn(av);
                 }
-                __threadfence();
                 __syncwarp();
-                if (lane == 0) atomicAdd(p.done_gu + u, 1);
+                if (lane == 0) {
+                    __threadfence();  // the warp's stores, then the count
+                    atomicAdd(p.done_gu + u, 1);
+                }
             }
             group_sync(gi);  // the reduction scratch is free again
         } else {

@@ -94,17 +94,17 @@ __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int
 }
 
 // ============================================================== router
-// CTA: 4 warps; warp owns EE experts, lanes are the 32 residue classes of the
-// fixed order; TT tokens per CTA staged in smem as fp32 in the same
-// lane-interleaved layout as the weights: xs[tt][s4][lane] = float4 of
-// x[128*s4 + 32*j + lane], j = 0..3.
+// CTA: NW warps (8 for decode batches, 4 above); warp owns EE experts, lanes
+// are the 32 residue classes of the fixed order; TT tokens per CTA staged in
+// smem as fp32 in the same lane-interleaved layout as the weights:
+// xs[tt][s4][lane] = float4 of x[128*s4 + 32*j + lane], j = 0..3.
 // Optional side outputs for the fused decode kernel that follows: x16 (fp16
 // copy of x, written by the CTAs of expert block 0), nzero ints zeroed, and
 // the top-k picks: with tok_done set, the last CTA to finish a token group
 // (a counter per group, reset by that CTA) runs the top-k of its tokens and
 // writes idx / wout, so the next kernel reads T k picks, not T E logits.
-template <int TT, int EE, int CH>
-__global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__restrict__ x, int T,
+template <int TT, int EE, int CH, int NW>
+__global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__restrict__ x, int T,
                                                      int H, const float4 *__restrict__ Wp,
                                                      const float *__restrict__ bias, int E,
                                                      float *__restrict__ logits,
@@ -123,7 +123,7 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
     const bool write16 = x16 != nullptr && blockIdx.x == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e0 = (blockIdx.x * 4 + warp) * EE;
+    const int e0 = (blockIdx.x * NW + warp) * EE;
     // the first CH steps of this warp's weights are requested before the
     // token rows are staged, so the two latencies overlap
     float4 wv[CH][EE];
@@ -236,7 +236,7 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
     __syncthreads();
     if (!s_last) return;
     __threadfence();  // every CTA's logits of this token group are visible
-    for (int a = warp; a < TT; a += 4) {
+    for (int a = warp; a < TT; a += NW) {
         const int t = t0 + a;
         if (t >= T) break;
         int pe;
@@ -250,14 +250,14 @@ __global__ __launch_bounds__(128) void router_kernel(const __nv_bfloat16 *__rest
     if (threadIdx.x == 0) tok_done[blockIdx.y] = 0;  // ready for the next launch
 }
 
-template <int TT, int EE, int CH>
+template <int TT, int EE, int CH, int NW>
 static void run_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
                        float *logits, void *x16, int *zero, int nzero, int k, int32_t *idx,
                        float *w, int *tok_done, cudaStream_t s) {
     size_t smem = (size_t)TT * H * sizeof(float);
-    auto kern = router_kernel<TT, EE, CH>;
-    dim3 grid((E + 4 * EE - 1) / (4 * EE), (T + TT - 1) / TT);
-    kern<<<grid, 128, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
+    auto kern = router_kernel<TT, EE, CH, NW>;
+    dim3 grid((E + NW * EE - 1) / (NW * EE), (T + TT - 1) / TT);
+    kern<<<grid, 32 * NW, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
                                  reinterpret_cast<const float4 *>(Wp), bias, E, logits,
                                  reinterpret_cast<__half *>(x16), zero, nzero, k, idx, w,
                                  tok_done);
@@ -267,13 +267,13 @@ void launch_router(const void *x, int T, int H, const float *Wp, const float *bi
                    float *logits, cudaStream_t s, void *x16, int *zero, int nzero, int k,
                    int32_t *idx, float *w, int *tok_done) {
     if (T <= 1)
-        run_router<1, 1, 20>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<1, 1, 20, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 4)
-        run_router<4, 1, 20>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<4, 1, 20, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 64)
-        run_router<8, 2, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<8, 2, 8, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else
-        run_router<8, 8, 2>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<8, 8, 2, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
 }
 
 // ============================================================== top-k
@@ -795,10 +795,10 @@ void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, 
 
 cudaError_t route_init_attributes(int max_smem) {
     cudaError_t e;
-    if ((e = allow_max_dyn_smem(router_kernel<1, 1, 20>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<4, 1, 20>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<8, 2, 8>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<8, 8, 2>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<1, 1, 20, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<4, 1, 20, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<8, 2, 8, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<8, 8, 2, 4>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(route_small_kernel, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(screen_topk_kernel, max_smem)) != cudaSuccess) return e;
     return allow_max_dyn_smem(dispatch_count_kernel, max_smem);
