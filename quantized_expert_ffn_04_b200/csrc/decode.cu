@@ -37,8 +37,8 @@
 
 namespace strata {
 
-constexpr int kFWarps = 16;                     // compute warps: 4 groups of 4
-constexpr int kFGroups = 4;
+constexpr int kFGroups = 4;                     // compute groups of 4 warps
+constexpr int kFWarps = 4 * kFGroups;
 constexpr int kFThreads = 32 * (kFWarps + 1);   // + the copy warp
 constexpr int kFTile = 8;                       // tokens per unit (mma N)
 constexpr int kFMaxRing = 6;
@@ -291,18 +291,26 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     for (int i = tid; i < Tk; i += blockDim.x) atomicOr(&mask[sidx[i]], 1ull << (i / k));
     __syncthreads();
     // one scan of (count << 16 | units): both sums stay below 2^16 (T k <= 1024)
+    // thread tid owns experts [tid ept, tid ept + ept) (E <= 2 blockDim.x)
+    const int ept = (E + blockDim.x - 1) / blockDim.x, eb = tid * ept;
+    int local = 0;
+    for (int e = eb; e < eb + ept && e < E; e++) {
+        const int c = __popcll(mask[e]);
+        local += (c << 16) | ((c + kFTile - 1) / kFTile);
+    }
     int packed_total;
-    const int cnt = tid < E ? __popcll(mask[tid]) : 0;  // E <= blockDim.x
-    const int nu = (cnt + kFTile - 1) / kFTile;
-    const int packed = cta_exclusive_scan((cnt << 16) | nu, misc + kMiscScan, &packed_total);
-    const int off = packed >> 16, us = packed & 0xffff, utot = packed_total & 0xffff;
+    int packed = cta_exclusive_scan(local, misc + kMiscScan, &packed_total);
+    const int utot = packed_total & 0xffff;
     const int nsh = (T + kFTile - 1) / kFTile;
-    if (tid < E) {
-        soff[tid] = off;
+    for (int e = eb; e < eb + ept && e < E; e++) {
+        const int c = __popcll(mask[e]), nu = (c + kFTile - 1) / kFTile;
+        const int off = packed >> 16, us = packed & 0xffff;
+        soff[e] = off;
         for (int i = 0; i < nu; i++) {
-            const int n = cnt - i * kFTile;
-            units[nsh + us + i] = make_int4(tid, off + i * kFTile, n < kFTile ? n : kFTile, 0);
+            const int n = c - i * kFTile;
+            units[nsh + us + i] = make_int4(e, off + i * kFTile, n < kFTile ? n : kFTile, 0);
         }
+        packed += (c << 16) | nu;
     }
     if (tid < nsh) {
         const int n = T - tid * kFTile;
@@ -542,7 +550,7 @@ static int g_fused_max_smem = 0;
 static int g_fused_sms = 0;
 
 int fused_decode_supported(const Geometry &g, int T) {
-    return T >= 1 && T <= kFMaxT && g.E <= 512 && g.E <= kFThreads && g.k <= kFMaxK &&
+    return T >= 1 && T <= kFMaxT && g.E <= 512 && g.E <= 2 * kFThreads && g.k <= kFMaxK &&
            g.H % 128 == 0 && g.Ip % 128 == 0 && g.H <= 8192;
 }
 
