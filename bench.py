@@ -444,7 +444,7 @@ def run_own(args, wl):
     line = {
         "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": wl, "description": desc, "tokens_per_batch": T,
                    "hidden": shape.hidden, "experts": shape.n_experts, "top_k": shape.top_k,
@@ -452,7 +452,10 @@ def run_own(args, wl):
                    "l2": "inputs larger than L2: steps rotate over %d layers (%.1f GB of "
                          "expert weights)" % (NL, NL * (shape.n_experts + 1)
                                               * shape.expert_bytes / 1e9),
-                   "cuda_graphs": True, "parallelism": f"replicas x{world}"},
+                   "cuda_graphs": True, "parallelism": f"replicas x{world}",
+                   "arithmetic": "fp16 tensor-core operands with fp32 accumulation (decode: exact "
+                                 "small-integer weights x fp16 tokens; prefill: fp16 dequantised "
+                                 "weights), fp32 router, bf16 input and output"},
         "roofline": roof,
         "stages_ms": stage_ms,
         "step_bytes": statistics.mean(step_bytes),
