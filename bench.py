@@ -46,7 +46,13 @@ WORKLOADS = {
     "prefill-t8192": (gen.FLASH2, 8192, "Flash-Next-shaped MoE layer, prefill chunk T=8192, "
                                         "2-bit block-32"),
     "tiny-t8": (gen.TINY, 8, "tiny MoE layer H256 E16 k2 I64, T=8"),
+    # 48-layer expert stack: h <- h + MoE(RMSNorm(h)) through 48 resident layers
+    "stack48-t4": (gen.FLASH2, 4, "48-layer Flash-Next-shaped expert stack (~37 GB of 2-bit "
+                                  "experts resident), decode T=4"),
+    "stack48-t8192": (gen.FLASH2, 8192, "48-layer Flash-Next-shaped expert stack (~37 GB of "
+                                        "2-bit experts resident), prefill chunk T=8192"),
 }
+STACK_LAYERS = 48
 DEFAULT_WORKLOAD = "decode-t4"
 STAGES = ["router", "topk", "dispatch", "gateup", "down", "combine"]
 TIMING_NOTE = ("CUDA events recorded by the library on the launching stream around the kernel, "
@@ -194,6 +200,7 @@ def run_reference(args, wl):
     if rank != 0:
         return
     shape, T, desc = WORKLOADS[wl]
+    stack = wl.startswith("stack")  # a stack step passes every token through 48 layers
     n_layers = min(args.layers, 4)
     layers = [gen.layer_weights(shape, seed=0, layer=l) for l in range(n_layers)]
     xs = [gen.hidden(T, shape.hidden, seed=100, layer=l) for l in range(n_layers)]
@@ -225,9 +232,10 @@ def run_reference(args, wl):
     with ThreadPoolExecutor(cores) as ex:
         list(ex.map(step, range(args.steps)))
     dt = time.perf_counter() - t0
-    value = done[0] / dt
+    value = done[0] / dt / (STACK_LAYERS if stack else 1)
     line = {
-        "impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": "48-layer-stack tokens/s" if stack else "MoE-layer tokens/s",
+        "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": done[0], "steps_requested": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1000 / max(done[0], 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -480,6 +488,170 @@ def run_own(args, wl):
         dist.destroy_process_group()
 
 
+def run_stack(args, wl):
+    """One step = one pass of T tokens through the 48-layer stack
+    (strata_moe_stack_forward: RMSNorm, MoE layer, residual, per layer), each
+    step a CUDA graph that first restores the stack input."""
+    import torch
+    import quantized_expert_ffn_04_b200 as qe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.cuda.current_device()
+    shape, T, desc = WORKLOADS[wl]
+    NL = STACK_LAYERS
+    peaks, peak_kind = load_peaks()
+    # layer 0's workspace serves the whole stack; the others need only their weights
+    layers, host_layers = [], []
+    for l in range(NL):
+        hw = gen.layer_weights(shape, seed=0, layer=l)
+        layers.append(qe.Layer(hw, max_tokens=T if l == 0 else 8, device=dev))
+        if l < 2:
+            host_layers.append(hw)
+        del hw
+    handles = [L.handle for L in layers]
+    x0 = gen.hidden(T, shape.hidden, seed=200 + rank)
+    h0 = torch.from_numpy(x0.view(np.int16).copy()).view(torch.bfloat16).cuda()
+    h = torch.empty_like(h0)
+    trace = torch.empty((NL, T, shape.hidden), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    # distinct experts per layer on the stack's own inputs (for the step bytes)
+    h.copy_(h0)
+    qe.strata_moe_stack_forward(handles, h.data_ptr(), T, trace.data_ptr(), stream.cuda_stream)
+    layers[0].sync_status(stream)
+    distinct = []
+    if T <= 8:
+        xn = torch.empty_like(h0)
+        for l in range(NL):
+            # the layer routes RMSNorm of its input
+            qe.strata_moe_rmsnorm(trace[l].data_ptr(), xn.data_ptr(), T, shape.hidden,
+                                  stream.cuda_stream)
+            idx, _, _, _ = layers[l].route(xn)
+            distinct.append(int(torch.unique(idx).numel()))
+    torch.cuda.synchronize()
+
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        h.copy_(h0)
+        qe.strata_moe_stack_forward(handles, h.data_ptr(), T, None, cap.cuda_stream)
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    layers[0].sync_status(stream)
+    if dist:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clocks:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    layers[0].sync_status(stream)
+    ms = reduce_max(t0.elapsed_time(t1), dist, "cuda")
+    ms_step = ms / args.steps
+    value = weak_scaling_value(T * args.steps, world, ms)
+
+    # e2e: host buffers in and out around each pass (pinned)
+    hh = torch.from_numpy(x0.view(np.int16).copy()).pin_memory()
+    ho = torch.empty_like(hh).pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        h.view(torch.int16).copy_(hh, non_blocking=True)
+        qe.strata_moe_stack_forward(handles, h.data_ptr(), T, None, stream.cuda_stream)
+        ho.copy_(h.view(torch.int16), non_blocking=True)
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    layers[0].sync_status(stream)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dist, "cuda")
+    e2e_value = weak_scaling_value(T * e2e_steps, world, e2e_ms)
+
+    decode = T <= 64
+    if decode:
+        step_bytes = sum((d + 1) * shape.expert_bytes + shape.n_experts * shape.hidden * 4
+                         for d in distinct)
+        achieved = step_bytes / (ms_step / 1000.0) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "kernel": "whole 48-layer step (router + fused decode kernel "
+                "+ RMSNorm per layer)", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind + " hbm copy", "traffic": None,
+                "algorithmic_bytes_per_launch": step_bytes,
+                "launch_ms": ms_step, "timing": "CUDA events around the timed graph replays"}
+    else:
+        ip = (shape.inter + 127) // 128 * 128
+        flops = NL * 2.0 * 3 * shape.hidden * ip * T * (shape.top_k + 1)
+        achieved = flops / (ms_step / 1000.0) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roof = {"bound": "tensor", "kernel": "whole 48-layer step (expert GEMMs, router, "
+                "dispatch, combine, RMSNorm per layer)", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": peak_kind + " bf16 sustained (fp16 runs at the bf16 rate)",
+                "traffic": None, "algorithmic_flops_per_launch": flops,
+                "launch_ms": ms_step, "timing": "CUDA events around the timed graph replays"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cores = os.cpu_count() or 1
+        xs_host = [gen.hidden(T, shape.hidden, seed=200, layer=l) for l in range(2)]
+        v, n, dt = oracle_throughput(host_layers, xs_host, shape, args.cpu_budget, cores)
+        cpu = {"value": v / NL, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} (layer, token) forwards (routing + 11 experts each) over 2 "
+                         f"layers in {dt:.1f} s, divided by {NL} layers per stack pass"}
+    clk = clocks.summary()
+    per_layer = qe.strata_moe_launch_count(handles[0], T) + 1  # + RMSNorm
+    line = {
+        "metric": "48-layer-stack tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": wl, "description": desc, "tokens_per_batch": T,
+                   "hidden": shape.hidden, "experts": shape.n_experts, "top_k": shape.top_k,
+                   "inter": shape.inter, "bits": shape.bits, "layers": NL,
+                   "l2": "inputs larger than L2: each step reads the experts of 48 layers "
+                         "(%.1f GB resident)" % (NL * (shape.n_experts + 1)
+                                                 * shape.expert_bytes / 1e9),
+                   "cuda_graphs": True, "parallelism": f"replicas x{world}",
+                   "arithmetic": "fp16 tensor-core operands with fp32 accumulation, fp32 "
+                                 "router and RMSNorm, bf16 residual stream"},
+        "roofline": roof,
+        "distinct_experts": statistics.mean(distinct) if distinct else None,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.hidden * 2,
+                "d2h_bytes_per_step": T * shape.hidden * 2, "steps": e2e_steps},
+        "gpu_launches": per_layer * NL * args.steps,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                   "reasons": clk["reasons"], "samples": clk["samples"]},
+    }
+    del g
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -497,6 +669,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args, args.workload)
+    elif args.workload.startswith("stack"):
+        run_stack(args, args.workload)
     else:
         run_own(args, args.workload)
 
