@@ -73,6 +73,12 @@ class LayerShape:
 TINY = LayerShape(hidden=256, n_experts=16, top_k=2, inter=64, bits=2, router_bias=False)
 FLASH2 = LayerShape(hidden=2560, n_experts=512, top_k=10, inter=640, bits=2, router_bias=True)
 FLASH3 = LayerShape(hidden=2560, n_experts=512, top_k=10, inter=640, bits=3, router_bias=True)
+# the pruned 256-expert build of the same layer ("Strata Runs 125B
+# Qwen3.8-Flash-Next on a 12GB Gaming GPU at Up to 94 Tokens/s", section "The
+# Coder build: half the experts, most of the skill"); synthetic weights, and
+# how the experts are chosen is not on the path
+PRUNED256 = LayerShape(hidden=2560, n_experts=256, top_k=10, inter=640, bits=2,
+                       router_bias=True)
 STACK_LAYERS = 48
 
 

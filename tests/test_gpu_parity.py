@@ -7,7 +7,10 @@ fp64 layer output.  Workloads: the tiny layer (H 256, E 16, k 2, I 64, T 8), the
 Flash-Next-shaped layer (H 2560, E 512, k 10, I 640; the pages' shape: "Strata
 Runs 125B Qwen3.8-Flash-Next on a 12GB Gaming GPU at Up to 94 Tokens/s",
 section "What it is") at decode T = 1, 4 (2-bit), T = 64 (3-bit) and prefill
-T = 8192 (2-bit, sampled outputs), plus ragged and degenerate cases.
+T = 8192 (2-bit, sampled outputs), the pruned 256-expert build of the same
+layer ("Strata Runs 125B Qwen3.8-Flash-Next on a 12GB Gaming GPU at Up to 94
+Tokens/s", section "The Coder build: half the experts, most of the skill"), plus
+ragged and degenerate cases.
 """
 import numpy as np
 import pytest
@@ -64,6 +67,8 @@ CASES = [
     ("flash2-T4", gen.FLASH2, 4),
     ("flash2-T13", gen.FLASH2, 13),
     ("flash3-T64", gen.FLASH3, 64),
+    ("pruned256-T4", gen.PRUNED256, 4),
+    ("pruned256-T300", gen.PRUNED256, 300),
 ]
 
 
