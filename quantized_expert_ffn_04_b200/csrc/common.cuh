@@ -141,9 +141,42 @@ STRATA_DEV void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *b
         : "memory");
 }
 
+// L2 policy for data read once per forward (expert and router weights):
+// evict first, so the weight streams do not push the kernels' code, the
+// routing data and the activations out of L2 between launches.
+STRATA_DEV uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+STRATA_DEV void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                              uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// Read-only 16-byte load with an L2 cache policy (data constant for the kernel).
+STRATA_DEV float4 ldg_f4_hint(const float4 *p, uint64_t pol) {
+    float4 v;
+    asm("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+        : "l"(p), "l"(pol));
+    return v;
+}
+
 // Programmatic dependent launch: block until the preceding kernel in the
 // stream has completed and its memory is visible (a no-op when the kernel was
 // launched without the programmatic-serialization attribute).
+// gpu-scope add with acquire-release ordering (PTX memory model): its
+// release half is cumulative over the stores a preceding barrier ordered
+// first, its acquire half covers the loads a following barrier orders after.
+STRATA_DEV int atom_add_acq_rel_gpu(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 STRATA_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Let the next kernel of the stream start launching once every CTA of this
 // grid has called this (or exited).

@@ -378,15 +378,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                     const uint8_t *wg = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
                                         (size_t)slab * gu_bytes;
                     mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * gu_bytes));
-                    bulk_g2s(dst, wg, (uint32_t)gu_bytes, &full[slot]);
-                    bulk_g2s(dst + gu_bytes, wg + p.mat_bytes, (uint32_t)gu_bytes, &full[slot]);
+                    const uint64_t pol = l2_evict_first_policy();  // weights: read once
+                    bulk_g2s_hint(dst, wg, (uint32_t)gu_bytes, &full[slot], pol);
+                    bulk_g2s_hint(dst + gu_bytes, wg + p.mat_bytes, (uint32_t)gu_bytes, &full[slot],
+                                  pol);
                 } else {
                     const int di = item - N1, u = di / ndn, rg = di % ndn;
                     const int e = units[u].x;
                     const uint8_t *wd = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
                                         2 * p.mat_bytes + (size_t)rg * dn_bytes;
                     mbar_arrive_expect_tx(&full[slot], (uint32_t)dn_bytes);
-                    bulk_g2s(dst, wd, (uint32_t)dn_bytes, &full[slot]);
+                    bulk_g2s_hint(dst, wd, (uint32_t)dn_bytes, &full[slot],
+                                  l2_evict_first_policy());
                 }
             }
             // the CTA must not exit with copies in flight (abort path)

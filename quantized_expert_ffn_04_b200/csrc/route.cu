@@ -35,11 +35,41 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// Best of a lane's 16 entries: the largest key, and on equal keys the lowest
+// q.  A pairwise tree over adjacent entries: the left operand of every
+// comparison holds the lower q's, so ">=" keeps ties on the lower q.
+__device__ __forceinline__ void lane_best(const uint32_t (&key)[16], uint32_t &bk, int &bq) {
+    uint32_t k8[8], k4[4], k2[2];
+    int q8[8], q4[4], q2[2];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const bool l = key[2 * i] >= key[2 * i + 1];
+        k8[i] = l ? key[2 * i] : key[2 * i + 1];
+        q8[i] = l ? 2 * i : 2 * i + 1;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const bool l = k8[2 * i] >= k8[2 * i + 1];
+        k4[i] = l ? k8[2 * i] : k8[2 * i + 1];
+        q4[i] = l ? q8[2 * i] : q8[2 * i + 1];
+    }
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        const bool l = k4[2 * i] >= k4[2 * i + 1];
+        k2[i] = l ? k4[2 * i] : k4[2 * i + 1];
+        q2[i] = l ? q4[2 * i] : q4[2 * i + 1];
+    }
+    const bool l = k2[0] >= k2[1];
+    bk = l ? k2[0] : k2[1];
+    bq = l ? q2[0] : q2[1];
+}
+
 // Top-k of one token by one warp (E <= 512: lane l holds logits l, l+32, ...).
 // Each round takes the largest key over the warp (redux.sync max) and, among
 // the lanes holding it, the lowest expert id (redux.sync min), i.e. the larger
-// logit and on equal logits the lower id; the winning lane drops that entry.
-// Lane j < k ends with pick j and its weight exp(l_j - m) / sum.
+// logit and on equal logits the lower id; the winning lane drops that entry
+// and finds its next best.  Lane j < k ends with pick j and its weight
+// exp(l_j - m) / sum.
 __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
                                         int &pick_e, float &pick_w) {
     uint32_t key[16];
@@ -49,15 +79,9 @@ __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int
         const int e = q * 32 + lane;
         key[q] = (q < nq && e < E) ? logit_key(__ldcg(row + e)) : 0u;
     }
-    // this lane's best entry: largest key, then lowest q (= lowest id)
-    uint32_t bk = 0u;
-    int bq = 0;
-#pragma unroll
-    for (int q = 15; q >= 0; q--) {
-        const bool t = key[q] >= bk && key[q] != 0u;
-        bk = t ? key[q] : bk;
-        bq = t ? q : bq;
-    }
+    uint32_t bk;
+    int bq;
+    lane_best(key, bk, bq);
     uint32_t my_k = 0u;
     int my_e = -1;
     for (int j = 0; j < k; j++) {
@@ -68,20 +92,12 @@ __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int
             my_k = wk;
             my_e = (int)we;
         }
-        // the winning lane drops the entry and finds its next best
-        const bool mine = (int)(we & 31u) == lane;
-        const int wq = (int)(we >> 5);
-        uint32_t nk = 0u;
-        int nb = 0;
+        if ((int)(we & 31u) == lane) {
+            const int wq = (int)(we >> 5);
 #pragma unroll
-        for (int q = 15; q >= 0; q--) {
-            key[q] = (mine && q == wq) ? 0u : key[q];
-            const bool t = key[q] >= nk && key[q] != 0u;
-            nk = t ? key[q] : nk;
-            nb = t ? q : nb;
+            for (int q = 0; q < 16; q++) key[q] = q == wq ? 0u : key[q];
+            lane_best(key, bk, bq);
         }
-        bk = mine ? nk : bk;
-        bq = mine ? nb : bq;
     }
     const float my_v = key_logit(my_k);
     const float m = __shfl_sync(0xffffffffu, my_v, 0);
@@ -94,10 +110,11 @@ __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int
 }
 
 // ============================================================== router
-// CTA: NW warps (8 for decode batches, 4 above); warp owns EE experts, lanes
-// are the 32 residue classes of the fixed order; TT tokens per CTA staged in
-// smem as fp32 in the same lane-interleaved layout as the weights:
-// xs[tt][s4][lane] = float4 of x[128*s4 + 32*j + lane], j = 0..3.
+// CTA: NW warps; warp owns EE experts, lanes are the 32 residue classes of the
+// fixed order; TT tokens per CTA staged in shared memory as bf16 in the same
+// lane-interleaved layout as the weights: xs[tt][s4][lane] holds the 4 values
+// x[128*s4 + 32*j + lane], j = 0..3 (8 bytes, so the staging stores and the
+// LDS.64 reads are conflict-free; widening bf16 to fp32 is exact).
 // Optional side outputs for the fused decode kernel that follows: x16 (fp16
 // copy of x, written by the CTAs of expert block 0), nzero ints zeroed, and
 // the top-k picks: with tok_done set, the last CTA to finish a token group
@@ -113,7 +130,7 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
                                                      int32_t *__restrict__ idx,
                                                      float *__restrict__ wout,
                                                      int *__restrict__ tok_done) {
-    extern __shared__ float4 xs[];
+    extern __shared__ uint2 xs[];
     // a dependent kernel may be scheduled now; it waits for this grid's
     // completion before reading anything written here
     grid_launch_dependents();
@@ -127,52 +144,47 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
     // the first CH steps of this warp's weights are requested before the
     // token rows are staged, so the two latencies overlap
     float4 wv[CH][EE];
+    const uint64_t pol = l2_evict_first_policy();  // the weights are read once
     auto load_w = [&](int s0) {
 #pragma unroll
         for (int c = 0; c < CH; c++)
 #pragma unroll
             for (int b = 0; b < EE; b++) {
                 int e = e0 + b, s4 = s0 + c;
-                wv[c][b] = (e < E && s4 < ns4) ? __ldg(Wp + ((size_t)e * ns4 + s4) * 32 + lane)
-                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                wv[c][b] = (e < E && s4 < ns4)
+                               ? ldg_f4_hint(Wp + ((size_t)e * ns4 + s4) * 32 + lane, pol)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
             }
     };
     load_w(0);
-    // stage TT token rows (16 bytes = 8 bf16 per chunk); each thread requests a
-    // batch of 8 chunks before storing any, so the loads overlap
-    const int nchunk = TT * H / 8;
-    float *xf = reinterpret_cast<float *>(xs);
-    for (int base = 0; base < nchunk; base += 8 * blockDim.x) {
-        uint4 v[8];
+    // stage TT token rows: a thread fills slots (tt, s4, l) from four 2-byte
+    // loads that are coalesced across the warp; kSB slots (all of them for
+    // H = 2560 and TT <= 8) are requested per thread before any is stored,
+    // so the staging costs one memory round trip
+    constexpr int kSB = (TT * 20 + NW - 1) / NW < 20 ? (TT * 20 + NW - 1) / NW : 20;
+    const int nslot = TT * ns4 * 32;
+    const unsigned short *xu = reinterpret_cast<const unsigned short *>(x);
+    for (int base = 0; base < nslot; base += kSB * blockDim.x) {
+        uint32_t v[kSB][4];
 #pragma unroll
-        for (int b = 0; b < 8; b++) {
-            const int idx = base + b * blockDim.x + threadIdx.x;
-            v[b] = make_uint4(0, 0, 0, 0);
-            if (idx < nchunk) {
-                const int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
-                if (t0 + tt < T) v[b] = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H + i0);
-            }
+        for (int b = 0; b < kSB; b++) {
+            const int sl = base + b * blockDim.x + threadIdx.x;
+            const int tt = sl / (ns4 * 32), r = sl % (ns4 * 32);
+            const bool ok = sl < nslot && t0 + tt < T;
+            const unsigned short *px = xu + (size_t)(t0 + tt) * H + (r >> 5) * 128 + (r & 31);
+#pragma unroll
+            for (int j = 0; j < 4; j++) v[b][j] = ok ? (uint32_t)__ldg(px + 32 * j) : 0u;
         }
 #pragma unroll
-        for (int b = 0; b < 8; b++) {
-            const int idx = base + b * blockDim.x + threadIdx.x;
-            if (idx >= nchunk) break;
-            const int tt = idx / (H / 8), i0 = (idx % (H / 8)) * 8;
-            const __nv_bfloat16 *pv = reinterpret_cast<const __nv_bfloat16 *>(&v[b]);
+        for (int b = 0; b < kSB; b++) {
+            const int sl = base + b * blockDim.x + threadIdx.x;
+            if (sl >= nslot) break;
+            xs[sl] = make_uint2(v[b][0] | (v[b][1] << 16), v[b][2] | (v[b][3] << 16));
+            const int tt = sl / (ns4 * 32), r = sl % (ns4 * 32);
             if (write16 && t0 + tt < T) {
-                uint4 o;
-                __half2 *h2 = reinterpret_cast<__half2 *>(&o);
+                __half *o = x16 + (size_t)(t0 + tt) * H + (r >> 5) * 128 + (r & 31);
 #pragma unroll
-                for (int q = 0; q < 4; q++)
-                    h2[q] = __floats2half2_rn(__bfloat162float(pv[2 * q]),
-                                              __bfloat162float(pv[2 * q + 1]));
-                *reinterpret_cast<uint4 *>(x16 + (size_t)(t0 + tt) * H + i0) = o;
-            }
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int i = i0 + q;
-                xf[(((size_t)tt * ns4 + (i >> 7)) * 32 + (i & 31)) * 4 + ((i >> 5) & 3)] =
-                    __bfloat162float(pv[q]);
+                for (int j = 0; j < 4; j++) o[32 * j] = __float2half_rn(__uint_as_float(v[b][j] << 16));
             }
         }
     }
@@ -194,13 +206,15 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
             if (s4 >= ns4) break;
 #pragma unroll
             for (int a = 0; a < TT; a++) {
-                float4 xv = xs[((size_t)a * ns4 + s4) * 32 + lane];
+                const uint2 xv = xs[((size_t)a * ns4 + s4) * 32 + lane];
+                const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+                const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
 #pragma unroll
                 for (int b = 0; b < EE; b++) {
-                    acc[a][b] = fmaf(xv.x, wv[c][b].x, acc[a][b]);
-                    acc[a][b] = fmaf(xv.y, wv[c][b].y, acc[a][b]);
-                    acc[a][b] = fmaf(xv.z, wv[c][b].z, acc[a][b]);
-                    acc[a][b] = fmaf(xv.w, wv[c][b].w, acc[a][b]);
+                    acc[a][b] = fmaf(x0, wv[c][b].x, acc[a][b]);
+                    acc[a][b] = fmaf(x1, wv[c][b].y, acc[a][b]);
+                    acc[a][b] = fmaf(x2, wv[c][b].z, acc[a][b]);
+                    acc[a][b] = fmaf(x3, wv[c][b].w, acc[a][b]);
                 }
             }
         }
@@ -230,12 +244,16 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
     }
     if (tok_done == nullptr) return;
     __shared__ int s_last;
-    __threadfence();
+    // One gpu-scope acquire-release add per CTA: its release half publishes
+    // the logits this CTA stored (the barrier before it orders every warp's
+    // stores first), and in the last CTA of the token group its acquire half,
+    // extended to the other warps by the barrier after it, makes every other
+    // CTA's logits visible to the loads of the top-k.
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(tok_done + blockIdx.y, 1) == (int)gridDim.x - 1;
+    if (threadIdx.x == 0)
+        s_last = atom_add_acq_rel_gpu(tok_done + blockIdx.y, 1) == (int)gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
-    __threadfence();  // every CTA's logits of this token group are visible
     for (int a = warp; a < TT; a += NW) {
         const int t = t0 + a;
         if (t >= T) break;
@@ -254,7 +272,7 @@ template <int TT, int EE, int CH, int NW>
 static void run_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
                        float *logits, void *x16, int *zero, int nzero, int k, int32_t *idx,
                        float *w, int *tok_done, cudaStream_t s) {
-    size_t smem = (size_t)TT * H * sizeof(float);
+    size_t smem = (size_t)TT * H * sizeof(__nv_bfloat16);
     auto kern = router_kernel<TT, EE, CH, NW>;
     dim3 grid((E + NW * EE - 1) / (NW * EE), (T + TT - 1) / TT);
     kern<<<grid, 32 * NW, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
@@ -267,9 +285,9 @@ void launch_router(const void *x, int T, int H, const float *Wp, const float *bi
                    float *logits, cudaStream_t s, void *x16, int *zero, int nzero, int k,
                    int32_t *idx, float *w, int *tok_done) {
     if (T <= 1)
-        run_router<1, 1, 20, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<1, 1, 20, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 4)
-        run_router<4, 1, 20, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<4, 1, 20, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else if (T <= 64)
         run_router<8, 2, 8, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
     else
@@ -795,8 +813,8 @@ void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, 
 
 cudaError_t route_init_attributes(int max_smem) {
     cudaError_t e;
-    if ((e = allow_max_dyn_smem(router_kernel<1, 1, 20, 8>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(router_kernel<4, 1, 20, 8>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<1, 1, 20, 4>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(router_kernel<4, 1, 20, 4>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(router_kernel<8, 2, 8, 8>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(router_kernel<8, 8, 2, 4>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(route_small_kernel, max_smem)) != cudaSuccess) return e;
