@@ -183,6 +183,43 @@ def test_forward_host_matches_device():
     assert np.array_equal(yd, yh)
 
 
+def test_forward_host_pinned():
+    # pinned (page-locked) host buffers, as a serving loop holds them: new
+    # contents in the same buffers, other buffers, another T and a path
+    # change all give the device forward's bits
+    shape = gen.FLASH2
+    L = gpu_layer(shape, 8)
+    s = torch.cuda.Stream()
+
+    def pinned(a):
+        return torch.from_numpy(a.view(np.int16).copy()).pin_memory()
+
+    xa, xb = pinned(gen.hidden(8, shape.hidden, seed=7)), pinned(gen.hidden(8, shape.hidden, seed=8))
+    ya, yb = torch.empty_like(xa).pin_memory(), torch.empty_like(xb).pin_memory()
+
+    def device_ref(xp, T):
+        xd = to_dev_bf16(xp.numpy().view(np.uint16)[:T])
+        return from_dev_bf16(L.forward(xd))
+
+    def host(xp, yp, T):
+        qe.strata_moe_forward_host(L.handle, xp.data_ptr(), T, yp.data_ptr(), s.cuda_stream)
+        return yp.numpy().view(np.uint16)[:T].copy()
+
+    for T in (4, 1):
+        for xp, yp in ((xa, ya), (xb, yb)):
+            first = host(xp, yp, T)
+            again = host(xp, yp, T)
+            assert np.array_equal(first, device_ref(xp, T)) and np.array_equal(again, first)
+    host(xa, ya, 4)
+    xa.copy_(pinned(gen.hidden(8, shape.hidden, seed=9)))
+    assert np.array_equal(host(xa, ya, 4), device_ref(xa, 4))
+    qe.strata_moe_set_option(L.handle, qe.STRATA_OPT_PATH, 1)  # the decode kernel chain
+    y_chain = host(xa, ya, 4)
+    qe.strata_moe_set_option(L.handle, qe.STRATA_OPT_PATH, 0)
+    assert np.array_equal(y_chain, device_ref(xa, 4))
+    assert np.array_equal(host(xa, ya, 4), y_chain)
+
+
 def test_zero_and_oversized_batches():
     shape = gen.TINY
     L = gpu_layer(shape, 8)
