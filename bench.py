@@ -299,9 +299,9 @@ def run_own(args, wl):
     # second set of graphs used only for the per-stage pass: event nodes between
     # kernels would also cut the programmatic-launch chain of the headline steps.
     decode = T <= 64
-    # the fused decode kernel (router + one layer kernel) brackets only two stages
-    fused = qe.strata_moe_launch_count(layers[0].handle, T) == 2
-    stages = [0, GATEUP] if fused else ([0, 1] if T <= 256 else [0, 2]) + [3, 4, 5]
+    # the fused decode layer is one kernel: its probe is the gate/up stage
+    fused = decode and qe.strata_moe_launch_count(layers[0].handle, T) == 1
+    stages = [GATEUP] if fused else ([0, 1] if T <= 256 else [0, 2]) + [3, 4, 5]
     ev_b = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(NL)]
     ev_e = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(NL)]
     for l in range(NL):
@@ -376,19 +376,22 @@ def run_own(args, wl):
     stage_ms = {STAGES[st]: statistics.mean(ev_b[l][st].elapsed_time(ev_e[l][st]) for l in ran)
                 for st in stages}
     if fused:
-        stage_ms["topk+dispatch+gateup+down+combine (fused)"] = stage_ms.pop("gateup")
+        stage_ms["router+topk+dispatch+gateup+down+combine (fused)"] = stage_ms.pop("gateup")
     elif T <= 256:
         stage_ms["topk+dispatch"] = stage_ms.pop("topk")
 
     # ---- roofline of the dominant kernel (gate/up + SwiGLU)
     gu_ms = statistics.mean(ev_b[l][GATEUP].elapsed_time(ev_e[l][GATEUP]) for l in ran)
     if decode and fused:
-        gu_work = statistics.mean((distinct[l] + 1) * shape.expert_bytes + 2 * T * shape.hidden * 2
-                                  for l in ran)
+        # the whole layer: router weight and bias, the distinct experts' packed
+        # weights (all three matrices) and the shared expert's, token rows in and out
+        gu_work = statistics.mean(shape.n_experts * shape.hidden * 4 + shape.n_experts * 4
+                                  + (distinct[l] + 1) * shape.expert_bytes
+                                  + 2 * T * shape.hidden * 2 for l in ran)
         achieved = gu_work / (gu_ms / 1000.0) / 1e9  # GB/s
         peak = float(peaks["hbm_gbs"])
-        roof = {"bound": "hbm", "kernel": "fused_decode_kernel (top-k, dispatch, gate/up, down, "
-                "combine)", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        roof = {"bound": "hbm", "kernel": "fused_decode_kernel (router, top-k, dispatch, gate/up, "
+                "down, combine)", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind + " hbm copy",
                 "traffic": traffic_from_profile(wl), "algorithmic_bytes_per_launch": gu_work,
                 "launch_ms": gu_ms, "timing": TIMING_NOTE}

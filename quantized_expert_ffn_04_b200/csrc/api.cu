@@ -86,9 +86,14 @@ struct strata_moe {
     // routed token rows in slot order, then (at row T * k) the fp16 copy of x
     void *xs = nullptr;
     float *dsplit = nullptr;  // [max_tokens][router_rows] screening GEMM output (T > 256)
-    // fused decode counters: [units (tile 8)], [max_tokens][H / 128], item queues [2]
+    // fused decode layer: grid barrier counter (monotonic), two counter sets
+    // (finished gate/up slabs per unit, finished down blocks per (token, row
+    // block)) used by alternate launches, token prescale exponents
+    unsigned long long *fused_bar = nullptr;
     int *fused_cnt = nullptr;
-    int *tok_groups = nullptr;  // router top-k counters (one per token group, self-resetting)
+    int fused_stride = 0, fused_tok = 0;
+    int *xex = nullptr;
+    float *fcorr = nullptr;  // [min(max_tokens, 64)][H / 32] block corrections of the fused layer
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
     // options
     int path = 0;
@@ -171,8 +176,12 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->xn = take(T * H * 2);
     h->xs = take(slots * H * 2);
     h->dsplit = (float *)take(T > (size_t)kSmallMaxT ? T * (size_t)h->router_rows * 4 : 0);
-    h->fused_cnt = (int *)take(((size_t)units + T * (H / 128) + 2) * 4);
-    h->tok_groups = (int *)take(64 * 4);
+    h->fused_tok = max_units(64, (int)k, (int)E, 8);
+    h->fused_stride = h->fused_tok + 64 * (int)(H / 128);
+    h->fused_bar = (unsigned long long *)take(8);
+    h->fused_cnt = (int *)take((size_t)2 * h->fused_stride * 4);
+    h->xex = (int *)take(T * 4);
+    h->fcorr = (float *)take((T < 64 ? T : 64) * (H / 32) * 4);
     return off;
 }
 
@@ -273,28 +282,40 @@ bool use_fused_path(strata_moe_t h, int T) {
     return h->path == 0 && T <= h->decode_max_t && fused_decode_supported(h->geo, T);
 }
 
-// Router (+ fp16 copy of x and zeroed counters), then the fused kernel.
+// The whole layer in one launch (router, top-k, dispatch, experts, combine).
 strata_status run_forward_fused(strata_moe_t h, const void *x, int T, void *y, bool residual,
                                 cudaStream_t s) {
     const Geometry &g = h->geo;
     if (!fused_decode_supported(g, T))
         return fail(STRATA_ERR_INVALID_ARG, "the fused decode kernel does not support T=%d", T);
-    const int umax = max_units(T, g.k, g.E, 8);
-    probe(h, kStRouter, true, s);
-    launch_router(x, T, g.H, h->router_wp, h->router_b, g.E, h->logits, s, x16_of(h, T),
-                  h->fused_cnt, umax + T * (g.H / 128) + 2, g.k, h->idx, h->wts, h->tok_groups);
-    probe(h, kStRouter, false, s);
     ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
+    FusedArgs fa{};
+    fa.x = x;
+    fa.router_wp = h->router_wp;
+    fa.router_b = h->router_b;
+    fa.w2 = 0.0f;
+    fa.logits = h->logits;
+    fa.idx = h->idx;
+    fa.wts = h->wts;
+    fa.x16 = x16_of(h, T);
+    fa.xex = h->xex;
+    fa.corr = h->fcorr;
+    fa.a = h->a;
+    fa.Y = (float *)h->Y;
+    fa.out = y;
+    fa.residual = residual;
+    fa.bar = h->fused_bar;
+    fa.cnt = h->fused_cnt;
+    fa.cnt_stride = h->fused_stride;
+    fa.cnt_tok = h->fused_tok;
+    fa.err = h->err;
+    fa.budget = h->budget;
     probe(h, kStGateUp, true, s);
-    cudaError_t ce = launch_fused_decode(g, w, h->idx, h->wts, x16_of(h, T), T, umax, h->a,
-                                         (float *)h->Y, y, residual, h->fused_cnt,
-                                         h->fused_cnt + umax,
-                                         h->fused_cnt + umax + T * (g.H / 128), h->err,
-                                         h->budget, s);
+    cudaError_t ce = launch_fused_decode(g, w, fa, T, s);
     probe(h, kStGateUp, false, s);
     if (ce != cudaSuccess)
         return fail(STRATA_ERR_CUDA, "fused decode kernel: %s", cudaGetErrorString(ce));
-    return check_launch("fused decode kernels");
+    return check_launch("fused decode kernel");
 }
 
 strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool residual,
@@ -365,7 +386,7 @@ int strata_moe_launch_count(strata_moe_t h, int T) {
     // copy, screening GEMM, screened top-k, 3 dispatch kernels.  Then gate/up +
     // down (the tensor-core path adds the slot-order row gather, and the fp16
     // token copy when T <= kSmallMaxT), and the combine.
-    if (use_fused_path(h, T)) return 2;  // router, fused layer kernel
+    if (use_fused_path(h, T)) return 1;  // the fused layer kernel
     const bool decode = use_decode_path(h, T);
     if (T <= kSmallMaxT) return 2 + (decode ? 2 : 4) + 1;
     return 6 + 3 + 1;
@@ -601,6 +622,10 @@ strata_status strata_moe_sync_status(strata_moe_t h, void *stream) {
     if (e) {
         *h->err_host = 0;
         cudaMemsetAsync(h->err, 0, 4, s);
+        // a launch that gave up may leave the fused layer's barrier counter and
+        // per-launch counters mid-count: start them over
+        cudaMemsetAsync(h->fused_bar, 0, 8, s);
+        cudaMemsetAsync(h->fused_cnt, 0, (size_t)2 * h->fused_stride * 4, s);
         cudaStreamSynchronize(s);
         return fail(STRATA_ERR_TIMEOUT, "a device-side wait gave up (code %d)", e);
     }

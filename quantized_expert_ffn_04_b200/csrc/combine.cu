@@ -9,6 +9,8 @@
 //            w[t][j] * Y[slot[t][j]], in fp32, rounded once to bf16.
 // Stack: h <- bf16(f32(h) + f32(out)); RMSNorm weight 1, eps 1e-6 with the
 // sum of squares in the router's fixed order.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -153,10 +155,14 @@ void launch_selftest_wait(int *err, long long budget, cudaStream_t s) {
 }
 
 cudaError_t init_kernel_attributes() {
+    // one set-up per device; create and the allocation-free routing may call
+    // this from different host threads at once
+    static std::mutex mu;
     static bool done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && done[dev]) return cudaSuccess;
     int max_smem = 0;
     e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);

@@ -20,10 +20,15 @@ namespace strata {
 //                     for fragment register r' = 4s + r (s = k-step of the block,
 //                     r = mma A register 0..3): half 0 at bits P..P+1, half 1 at
 //                     bits 16+P..16+P+1, with P = code_pos(bits, r'):
-//                       2-bit: P = 2, 4, 6, 8, 10, 12, 14, 0 for r' = 0..7, so
-//                              that r' = 0..3 come out of one mask (the code sits
-//                              in the fp16 mantissa at bit 2, 4, 6 or 8), r' = 4..6
-//                              after one shift by 8 and r' = 7 after a shift by 2;
+//                       2-bit: P = 2, 10, 4, 12, 6, 14, 8, 0 for r' = 0..7:
+//                              r' = 0, 2, 4, 6 come out of one mask each (the code
+//                              sits in the fp16 mantissa at bit 2, 4, 6, 8),
+//                              r' = 1, 3, 5 after one shift right by 8 and r' = 7
+//                              after one shift left by 8, so the two registers
+//                              of a k-step that share columns (r and r + 1, r
+//                              even) hold their codes at the same mantissa bit
+//                              (2 + 2 (r' >> 1)): columns 8h .. 8h + 7 of a block
+//                              all sit at bit 2 + 2h;
 //                       3-bit: P = 2r'.
 //                     Register r holds (row, col) pairs of the m16n8k16 A
 //                     fragment: r=0 (g, 2c|2c+1), r=1 (g+8, 2c|2c+1),
@@ -40,7 +45,8 @@ constexpr int kHiBytes = 256;
 constexpr int kScaleBytes = 128;
 
 __host__ __device__ constexpr int code_pos(int bits, int rp) {
-    return bits == 2 ? (rp < 7 ? 2 * rp + 2 : 0) : 2 * rp;
+    return bits == 2 ? ((rp & 1) ? (rp == 7 ? 0 : 2 * (rp >> 1) + 10) : 2 * (rp >> 1) + 2)
+                     : 2 * rp;
 }
 
 __host__ __device__ constexpr int unit_bytes(int bits) {
@@ -79,6 +85,12 @@ STRATA_DEV void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// `count` arrivals at once.
+STRATA_DEV void mbar_arrive_cnt(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
 STRATA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -87,6 +99,21 @@ STRATA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// try_wait that lets the thread sleep until the phase completes or about
+// `ns` nanoseconds pass (a waiting thread then issues no instructions that the
+// SM's other warps could use).
+STRATA_DEV bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
         : "memory");
     return ok != 0;
 }
@@ -408,8 +435,8 @@ STRATA_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
 
 // Register r' (0..7) of a 2-bit block word: fp16 pair of 2q - 3.
 STRATA_DEV uint32_t dq2_pair(uint32_t w, int rp) {
-    const uint32_t src = rp < 4 ? w : (rp < 7 ? (w >> 8) : (w << 2));
-    const int j = rp < 4 ? rp : (rp < 7 ? rp - 4 : 0);  // pe = 2 j + 2
+    const uint32_t src = (rp & 1) ? (rp == 7 ? (w << 8) : (w >> 8)) : w;
+    const int j = rp >> 1;  // the code sits at mantissa bit 2 j + 2
     const uint32_t mask = (3u << (2 * j + 2)) | (3u << (16 + 2 * j + 2));
     return hfma2_u32((src & mask) | 0x64006400u, dq2_mul(j), dq2_off(j));
 }
@@ -428,23 +455,23 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
         ".reg .f32 z;\n\t"
         "mov.f32 z, 0f00000000;\n\t"
         "shr.b32 s8, %4, 8;\n\t"
-        "shl.b32 s2, %4, 2;\n\t"
+        "shl.b32 s2, %4, 8;\n\t"
         "lop3.b32 h0, %4, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h1, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h2, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h3, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h4, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h5, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h6, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h7, s2, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h1, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h2, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h3, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h4, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h5, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h6, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h7, s2, 0x03000300, 0x64006400, 0xEA;\n\t"
         "fma.rn.f16x2 h0, h0, %9, %13;\n\t"
-        "fma.rn.f16x2 h1, h1, %10, %14;\n\t"
-        "fma.rn.f16x2 h2, h2, %11, %15;\n\t"
-        "fma.rn.f16x2 h3, h3, %12, %16;\n\t"
-        "fma.rn.f16x2 h4, h4, %9, %13;\n\t"
-        "fma.rn.f16x2 h5, h5, %10, %14;\n\t"
-        "fma.rn.f16x2 h6, h6, %11, %15;\n\t"
-        "fma.rn.f16x2 h7, h7, %9, %13;\n\t"
+        "fma.rn.f16x2 h1, h1, %9, %13;\n\t"
+        "fma.rn.f16x2 h2, h2, %10, %14;\n\t"
+        "fma.rn.f16x2 h3, h3, %10, %14;\n\t"
+        "fma.rn.f16x2 h4, h4, %11, %15;\n\t"
+        "fma.rn.f16x2 h5, h5, %11, %15;\n\t"
+        "fma.rn.f16x2 h6, h6, %12, %16;\n\t"
+        "fma.rn.f16x2 h7, h7, %12, %16;\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h0,h1,h2,h3}, "
         "{%5,%6}, {z,z,z,z};\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h4,h5,h6,h7}, "
@@ -454,6 +481,50 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
         : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(0x38003800u), "r"(0x30003000u),
           "r"(0x28002800u), "r"(0x20002000u), "r"(0xE006E006u), "r"(0xD818D818u),
           "r"(0xD060D060u), "r"(0xC980C980u));
+}
+
+// The same block without normalising the codes: each fragment register holds
+// h = 1024 + q 2^P (the code at mantissa bit P = 2 + 2 (r' >> 1), exact), and
+// the token operand carries the column group's factor: B_k = x_k 2^(8 - P_k)
+// for column k of the block (P_k = 2 + 2 ((k mod 32) >> 3)).  Then
+//   sum_k h_k B_k = sum_k 1024 B_k + 2^8 sum_k q_k x_k,
+// so with the accumulator started at c = -sum_k (1024 + 1.5 2^P_k) B_k (one
+// value per token column: c0 for column 2 (lane & 3), c1 for the next) the
+// result is 2^8 sum_k (q_k - 1.5) x_k, the block's dot product with the
+// dequantised weights over its scale, times 2^8.  Two shifts and 8 mask/or
+// per block, no packed fma.
+STRATA_DEV void block_mma2m(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, uint32_t b2,
+                            uint32_t b3, float c0, float c1) {
+    asm(
+        "{\n\t"
+        ".reg .b32 s8, s2, h0, h1, h2, h3, h4, h5, h6, h7;\n\t"
+        "shr.b32 s8, %4, 8;\n\t"
+        "shl.b32 s2, %4, 8;\n\t"
+        "lop3.b32 h0, %4, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h1, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h2, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h3, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h4, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h5, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h6, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h7, s2, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h0,h1,h2,h3}, "
+        "{%5,%6}, {%9,%10,%9,%10};\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h4,h5,h6,h7}, "
+        "{%7,%8}, {%0,%1,%2,%3};\n\t"
+        "}\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "f"(c0), "f"(c1));
+}
+
+// Column factor of the magic-offset token operand and the correction weight
+// of column k of a block (see block_mma2m), kk = k mod 32:
+// B_k = x_k * magic_col_scale(kk) = x_k 2^(8 - P_k), c_k = 1024 + 1.5 * 2^P_k.
+__host__ __device__ inline float magic_col_scale(int kk) {  // kk = k mod 32
+    return (float)(1 << (6 - 2 * (kk >> 3)));
+}
+__host__ __device__ inline float magic_col_corr(int kk) {
+    return 1024.0f + 1.5f * (float)(1 << (2 + 2 * (kk >> 3)));
 }
 
 // ---------------------------------------------------------------- GEMV blocks

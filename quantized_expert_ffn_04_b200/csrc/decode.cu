@@ -1,87 +1,141 @@
-// Fused decode layer (T <= 64 tokens): top-k, dispatch, gate/up + SwiGLU,
-// down and the combine in ONE persistent kernel that follows the router.
+// Fused decode layer (T <= 64 tokens): the whole mixture-of-experts layer in
+// ONE persistent kernel, one CTA per SM: router logits, top-k, dispatch,
+// gate/up + SwiGLU, down and the fixed-order combine.
 //
-// Layer specification (the same steps as the multi-kernel path): the router
-// kernel before it leaves the picks (the k largest logits, a tie to the lower
-// expert id) and w_j = exp(l_j - m) / sum over the picks; units = (expert, up
-// to 8 of its tokens), the shared
-// expert's units first; a = silu(Wg x) * Wu x, y = Wd a with w = d (q - c) from
-// the block-32 codes; out = y_shared + sum over the picks in ascending expert
-// id of w_j y_j (fp32), rounded once to bf16.  The pages: 10 routed + 1 shared
-// expert per token ("Strata Runs 125B Qwen3.8-Flash-Next on a 12GB Gaming GPU
-// at Up to 94 Tokens/s", section "What it is"), decode of one token or a small
-// multi-token-prediction batch (section "The numbers, measured by the author").
+// Layer specification (the same steps as the multi-kernel path):
+//   logit[t][e] = sum_i x[t][i] W[e][i] + b[e] in fp32 in the fixed order (32
+//   lane partials over i = l, l+32, ..., fma in ascending i, then a halving
+//   tree); picks = the k largest logits, a tie to the lower expert id;
+//   w_j = exp(l_j - m) / sum over the picks; units = (expert, up to 8 of its
+//   tokens), the shared expert's units first; a = silu(Wg x) * Wu x,
+//   y = Wd a with w = d (q - c) from the block-32 codes; out = y_shared + sum
+//   over the picks in ascending expert id of w_j y_j (fp32), rounded once to
+//   bf16.  The pages: 10 routed + 1 shared expert per token ("Strata Runs 125B
+//   Qwen3.8-Flash-Next on a 12GB Gaming GPU at Up to 94 Tokens/s", section
+//   "What it is"), routers and shared experts on the GPU (section "How a 125B
+//   model fits in 12 GB"), decode of one token or a small multi-token-
+//   prediction batch (section "The numbers, measured by the author").
 //
 // Why one kernel: at T = 1..4 the layer moves 20-55 MB, ~3-9 us of HBM time,
-// while each extra launch in a chain costs a few microseconds of ramp and
-// drain.  Here:
-//   * every CTA builds the dispatch tables itself (identical, deterministic)
-//     from the router's T k picks, so no grid-wide barrier;
-//   * each CTA owns a contiguous range of gate/up items (unit, 16-row slab)
-//     and then of down items (unit, 128 rows); a copy warp streams the
-//     items' packed weights through a ring of shared-memory slots with bulk
-//     copies, up to `ring` items ahead, while 4 groups of 4 warps compute;
-//   * a down item of unit u waits (bounded) until all gate/up slabs of u are
-//     done (a counter per unit); every CTA finishes its gate/up items before
-//     its down items, so the waits always end;
-//   * the down item that completes the last expert's rows of a (token,
-//     128-row block) pair (a counter per pair) combines that block of the
-//     token, in the fixed order, so the combine is spread over the down
-//     items instead of waiting for all of them.
-// The counters are zeroed by the router kernel, which this kernel waits for
-// (programmatic dependent launch).  The math of a block is the decode GEMV's:
-// exact small integers from the codes, fp16 token rows, mma.sync as the
-// in-warp reduction, fp32 per-block scaling.
+// so every dependent step costs as much as the traffic.  The structure:
+//   * warp roles: 16 compute warps (4 groups of 4), a copy warp that streams
+//     packed weights into a ring of shared-memory slots with 1-D bulk copies,
+//     a publish warp and a fetch warp (below);
+//   * prologue: the copy warp requests this CTA's slice of the router weight
+//     (E / #SMs experts) and, for T <= 8, the shared expert's gate/up slabs
+//     assigned to this CTA, before the previous kernel has finished
+//     (programmatic dependent launch): neither depends on routing;
+//   * router: each CTA computes the logits of its experts for every token;
+//     one grid-wide barrier (a monotonic counter, bounded waits; the launch
+//     is cooperative, so every CTA is resident) makes all logits visible;
+//     meanwhile the compute groups run the shared expert's gate/up slabs;
+//   * top-k and dispatch: every CTA runs them itself (identical and
+//     deterministic), for T > 16 tokens the top-k is split over CTAs with a
+//     second barrier;
+//   * items: the list [routed gate/up slabs (unit, 16 rows)] + [down blocks
+//     (unit, 128 rows)] is dealt out round-robin over the CTAs, so at every
+//     step all CTAs work on neighbouring units: a unit's gate/up slabs are
+//     all done long before its down blocks come up, and no item is claimed
+//     with an atomic;
+//   * two groups of 8 compute warps take alternate ring positions; the 8
+//     warps of a group each take a share of the item (an eighth of K of both
+//     the gate and the up slab; two slabs and half of K of a down block, so
+//     one token fragment serves two slabs) and run independently: no barrier
+//     inside the item loop, and a ring slot is free as soon as its last warp
+//     is done, so most of the ring is in flight; the last warp to finish an
+//     item completes it (sums the partial products in a fixed order and
+//     applies SwiGLU, or stores the block's rows and counts them for the
+//     combine);
+//   * the publish warp turns finished gate/up slabs into per-unit counts
+//     (one gpu-scope fence per batch), and the fetch warp waits for the
+//     counts a down block needs and copies that unit's activation rows in,
+//     so the compute warps never wait on a fence or a remote counter;
+//   * the down block that completes the last expert rows of a (token,
+//     128-row block) pair combines that block of the token in the fixed order.
+// The math of a block: mma.sync as the in-warp reduction with fp32 per-block
+// scaling.  Gate/up (2-bit) take the magic-offset form (block_mma2m: the codes
+// go into the fp16 mantissa with one mask each, and the constant offset is
+// taken out through the accumulator with a precomputed per-(token, block)
+// correction); the down blocks and the 3-bit weights use the exact small
+// integers 2q - (2^bits - 1).  Every wait is bounded; on expiry the CTA records a timeout in the
+// error word, lets its copies land and returns.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace strata {
 
-constexpr int kFGroups = 4;                     // compute groups of 4 warps
-constexpr int kFWarps = 4 * kFGroups;
-constexpr int kFThreads = 32 * (kFWarps + 1);   // + the copy warp
+constexpr int kFWarps = 16;                     // compute warps
+constexpr int kGroups = 2, kGWarps = 8;         // two groups of 8 take alternate ring positions
+constexpr int kFCompute = 32 * kFWarps;         // compute threads
+constexpr int kWCopy = kFWarps, kWPub = kFWarps + 1, kWFetch = kFWarps + 2, kWComb = kFWarps + 3;
+constexpr int kFThreads = 32 * (kFWarps + 4);
 constexpr int kFTile = 8;                       // tokens per unit (mma N)
-constexpr int kFMaxRing = 6;
-constexpr int kDownSlabs = 8;                   // a down item: 8 slabs = 128 rows
+constexpr int kFMaxRing = 8;
+constexpr int kDownSlabs = 8;                   // a down block: 8 slabs = 128 rows
 constexpr int kFStagedMaxT = 8;                 // token rows kept in shared memory
 constexpr int kFMaxT = 64;                      // most tokens per call
 constexpr int kFMaxK = 16;                      // most routed experts per token
+constexpr int kTopkLocalT = 16;                 // up to here every CTA runs the whole top-k
+constexpr int kPubQ = 64;                       // publish queue entries
+constexpr int kMaxA = 4;                        // activation buffers (one down block each)
+constexpr int kRedSlot = kGWarps * 32 * 8 * 4;  // partial sums of one ring slot (bytes)
+
+// item kinds in a ring slot's meta word
+constexpr int kItemEnd = -1;
+constexpr int kKindExtra = 1, kKindGU = 2, kKindDown = 3;
+__host__ __device__ inline int item_kind(int m) { return (m >> 28) & 7; }
 
 struct FusedParams {
+    const __nv_bfloat16 *x;   // [T][H] layer input
+    const float4 *Wp;         // router weight, [E][H/128][32 lanes] float4 (lane-interleaved)
+    const float *bias;        // [E] or null
     const uint8_t *routed;
     const uint8_t *shared;
     size_t expert_bytes, mat_bytes;
-    const int32_t *idx;    // [T][k] top-k picks (router)
-    const float *wts;      // [T][k] their weights (router)
-    const __half *x16;     // [T][H] fp16 copy of x (router)
     int T, E, k, H, Ip, nseg_h, nseg_i;
-    int ring, item_bytes, staged, units_max;
-    __half *a;             // [slots][Ip]
-    float *Y;              // [slots][H]
-    __nv_bfloat16 *out;    // [T][H]
+    int ring, item_bytes, staged, units_max, na;
+    float w2;                 // bound of every gate/up row's L2 norm (token prescale), 0: none
+    float *logits;            // [T][E]
+    int32_t *idx;             // [T][k] picks (T > kTopkLocalT: exchanged between CTAs)
+    float *wts;               // [T][k]
+    __half *x16;              // [T][H] fp16 token operand (T > kFStagedMaxT)
+    float *corr;              // [T][H / 32] its block corrections (T > kFStagedMaxT, 2-bit)
+    int *xex;                 // [T] token prescale exponents (T > kFStagedMaxT)
+    __half *a;                // [slots][Ip]
+    float *Y;                 // [slots][H] (scaled by 2^(-2 ex) of the token)
+    __nv_bfloat16 *out;       // [T][H]
     int residual;
-    int *done_gu;          // [units_max] finished gate/up slabs per unit
-    int *done_tok;         // [T][H / 128] finished down items per (token, row block)
-    int *queue;            // [2] next gate/up item, next down item (claimed by CTAs)
+    unsigned long long *bar;  // grid barrier counter, 2 arrivals per CTA per launch
+    int *cnt;                 // two counter sets of cnt_stride ints, used alternately
+    int cnt_stride;           // ints per set: finished gate/up slabs per unit, then
+    int cnt_tok;              // (at this offset) finished down blocks per (token, row block)
     int *err;
     long long budget;
 };
 
 // Shared-memory carve (host and device agree on it).
 struct FusedSmem {
-    int ring, xs, abuf, red, sidx, sw, sslot, sord, mask, soff, units, slist, misc, bars, total;
+    int ring, red, xs, corr, rega, sidx, sw, sslot, sord, mask, soff, units, slist, sex, misc,
+        bars, total;
 };
 
 __host__ __device__ inline int align16(int v) { return (v + 15) & ~15; }
+__host__ __device__ inline int imax(int a, int b) { return a > b ? a : b; }
 
 __host__ __device__ inline FusedSmem fused_smem(int T, int E, int k, int H, int Ip, int ring,
-                                                int item_bytes, int staged, int units_max) {
+                                                int item_bytes, int staged, int units_max,
+                                                int na) {
     FusedSmem s;
     int o = 0;
     s.ring = o;  o += ring * item_bytes;
+    // partial sums of the warps, per ring slot; while routing it holds the
+    // lane-interleaved bf16 copy of the token rows that the router reads
+    s.red = o;   o += ring * kRedSlot;
     s.xs = o;    o += staged ? align16(T * (H + 8) * 2) : 0;
-    s.abuf = o;  o += kFGroups * kFTile * (Ip + 8) * 2;  // a rows of each group's down item
-    s.red = o;   o += kFGroups * 4 * 32 * 8 * 4;
+    s.corr = o;  o += staged ? align16((H / 32) * kFTile * 4) : 0;
+    // the raw bf16 token rows while routing, then the activation buffers
+    s.rega = o;  o += imax(staged ? align16(T * H * 2) : 0, na * kFTile * (Ip + 8) * 2);
     s.sidx = o;  o += align16(T * k * 4);
     s.sw = o;    o += align16(T * k * 4);
     s.sslot = o; o += align16(T * k * 4);
@@ -90,15 +144,27 @@ __host__ __device__ inline FusedSmem fused_smem(int T, int E, int k, int H, int 
     s.soff = o;  o += align16(E * 4);
     s.units = o; o += units_max * 16;
     s.slist = o; o += align16(T * k * 4);
-    s.misc = o;  o += 512;                       // flags, scan scratch, combine lists, item ids
-    s.bars = o;  o += 8 * (2 * kFMaxRing + 2 + kFGroups);
+    s.sex = o;   o += align16(T * 4);
+    s.misc = o;  o += 256 * 4;
+    s.bars = o;  o += 8 * (2 * kFMaxRing + 8 + 2 * kMaxA);
     s.total = o;
     return s;
 }
 
-// Exclusive scan of one int per thread over the whole CTA (<= 32 warps).
-__device__ int cta_exclusive_scan(int v, int *scratch, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// misc ints
+constexpr int kMiscAbort = 0, kMiscScan = 1 /* 33 */, kMiscNUnits = 34, kMiscUtot = 35,
+              kMiscPar = 36, kMiscDead = 37, kMiscCFlag = 38, kMiscTmp = 39,
+              kMiscGCnt = 40 /* kFMaxRing: warps done with the item in a slot */,
+              kMiscMeta = 48 /* kFMaxRing */, kMiscPubN = 56, kMiscPubSeen = 57,
+              kMiscWarpsDone = 58, kMiscCombN = 59, kMiscCombSeen = 60,
+              kMiscPubQ = 64 /* kPubQ */, kMiscCombQ = 128 /* kPubQ */;
+
+// Named barrier 1: the compute warps.
+STRATA_DEV void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFCompute) : "memory"); }
+
+// Exclusive scan of one int per compute thread over the compute warps.
+__device__ int compute_exclusive_scan(int v, int *scratch, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -106,29 +172,29 @@ __device__ int cta_exclusive_scan(int v, int *scratch, int *total) {
         if (lane >= o) incl += n;
     }
     if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
+    compute_sync();
     if (warp == 0) {
-        int s = lane < nw ? scratch[lane] : 0, si = s;
+        int s = lane < kFWarps ? scratch[lane] : 0, si = s;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int n = __shfl_up_sync(0xffffffffu, si, o);
             if (lane >= o) si += n;
         }
-        if (lane < nw) scratch[lane] = si - s;
+        if (lane < kFWarps) scratch[lane] = si - s;
         if (lane == 31) scratch[32] = si;
     }
-    __syncthreads();
+    compute_sync();
     const int r = scratch[warp] + incl - v;
     *total = scratch[32];
-    __syncthreads();
+    compute_sync();
     return r;
 }
 
 // B fragment source of a 32-wide block at column k0 (mma m16n8k16, fp16):
 // lane 4g + c needs x[token g][k0 + 8m + 2c], x[..+1] in register m = 0..3.
-//   kSrcSmem:  the token rows staged in shared memory, fetched with one
-//              ldmatrix (rowp = this lane's row for matrix row lane & 7);
-//   kSrcLdg:   read-only global rows through L1 (rowp = row of token lane >> 2);
+//   kSrcSmem:  rows staged in shared memory, fetched with one ldmatrix
+//              (rowp = this lane's row for matrix row lane & 7);
+//   kSrcLdg:   read-only global rows through L1 (rowp = row of token lane >> 2).
 constexpr int kSrcSmem = 0, kSrcLdg = 1;
 
 template <int kSrc>
@@ -145,45 +211,77 @@ STRATA_DEV void b_frag(const __half *rowp, int k0, int lane, uint32_t &b0, uint3
     }
 }
 
-// acc0/acc1 (16 rows x 8 tokens fragments) += two slabs' segments [0, ns),
-// held in shared memory at w0 and w1, against the same token rows from rowp
-// starting at column col0: one B fragment per block serves both slabs, and
-// the two mma chains are independent.  Each lane reads its rows' four block
-// scales with one 16-byte load (lane 4g + c: scales of rows g and g + 8).
-template <int kBits, int kSrc>
-STRATA_DEV void fused_slab2(float (&acc0)[4], float (&acc1)[4], const uint8_t *w0,
-                            const uint8_t *w1, int ns, const __half *rowp, int col0, int lane) {
+// acc (16 rows x 8 token columns, fp32 fragment) += blocks [b0, b1) of one
+// 16-row slab held in shared memory at `slab` (units of 128 columns) against
+// the token rows from rowp.  kMagic: the 2-bit magic-offset form
+// (block_mma2m; the token operand carries the column factors, ca/cb give the
+// block corrections of the lane's two token columns, and acc comes out times
+// 2^8); otherwise the exact small integers 2q - (2^bits - 1) (acc times 2).
+// One block against the B fragment: dequantise (exact integers, or the
+// magic-offset form with the block corrections c0 / c1) and two mma.
+template <int kBits, bool kMagic>
+STRATA_DEV void block_dot(float (&d)[4], uint32_t lo, uint32_t hi, int hshift, uint32_t b0,
+                          uint32_t b1, uint32_t b2, uint32_t b3, float c0, float c1) {
+    if (kMagic)
+        block_mma2m(d, lo, b0, b1, b2, b3, c0, c1);
+    else if (kBits == 2)
+        block_mma2(d, lo, b0, b1, b2, b3);
+    else
+        block_mma<kBits>(d, lo, hi, hshift, b0, b1, b2, b3);
+}
+
+// acc0 / acc1 (16 rows x 8 token columns, fp32 fragments) += blocks [b0, b1)
+// of two 16-row slabs held in shared memory at s0 and s1 (units of 128
+// columns) against the same token rows from rowp: one B fragment per block
+// serves both slabs.  b0 is even, so every pair of blocks sits inside one
+// unit; blocks go four at a time with no branch between them (eight
+// independent mma chains), each pair's code words and scales coming in with
+// one 8-byte load per slab (lane 4g + c holds its code words; the scales of
+// rows g and g + 8).  kMagic: the 2-bit magic-offset form (block_mma2m; the
+// token operand carries the column factors, ca[b] / cb[b] are the block
+// corrections of the lane's two token columns, and the sums come out times
+// 2^8); otherwise the exact small integers 2q - (2^bits - 1) (sums times 2).
+template <int kBits, int kSrc, bool kMagic>
+STRATA_DEV void slab2_blocks(float (&acc0)[4], float (&acc1)[4], const uint8_t *s0,
+                             const uint8_t *s1, int b0, int b1, const __half *rowp,
+                             const float *ca, const float *cb, int lane) {
     constexpr int UB = unit_bytes(kBits);
     constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
     const int g = lane >> 2;
-    for (int sg = 0; sg < ns; sg++) {
-        const uint8_t *u0 = w0 + sg * UB, *u1 = w1 + sg * UB;
-        const uint4 lo0 = *reinterpret_cast<const uint4 *>(u0 + lane * 16);
-        const uint4 lo1 = *reinterpret_cast<const uint4 *>(u1 + lane * 16);
-        uint2 hi0 = make_uint2(0, 0), hi1 = make_uint2(0, 0);
-        if (kBits == 3) {
-            hi0 = *reinterpret_cast<const uint2 *>(u0 + kLoBytes + lane * 8);
-            hi1 = *reinterpret_cast<const uint2 *>(u1 + kLoBytes + lane * 8);
-        }
-        const uint4 sc0 = *reinterpret_cast<const uint4 *>(u0 + SOFF + g * 16);
-        const uint4 sc1 = *reinterpret_cast<const uint4 *>(u1 + SOFF + g * 16);
+    int b = b0;
+    for (; b + 4 <= b1; b += 4) {
+        uint2 lw[2][2], kw[2][2];   // [pair][slab]: code words, scale words
+        uint32_t hw[2][2];          // 3-bit: the high-bit word of each pair
 #pragma unroll
-        for (int blk = 0; blk < 4; blk++) {
-            uint32_t b0, b1, b2, b3;
-            b_frag<kSrc>(rowp, col0 + sg * 128 + blk * 32, lane, b0, b1, b2, b3);
-            float d0[4], d1[4];
-            if (kBits == 2) {
-                block_mma2(d0, comp4(lo0, blk), b0, b1, b2, b3);
-                block_mma2(d1, comp4(lo1, blk), b0, b1, b2, b3);
-            } else {
-                block_mma<kBits>(d0, comp4(lo0, blk), blk < 2 ? hi0.x : hi0.y, 8 * (blk & 1), b0,
-                                 b1, b2, b3);
-                block_mma<kBits>(d1, comp4(lo1, blk), blk < 2 ? hi1.x : hi1.y, 8 * (blk & 1), b0,
-                                 b1, b2, b3);
+        for (int pp = 0; pp < 2; pp++) {
+            const int bp = b + 2 * pp;
+            const int off = (bp >> 2) * UB, wo = (bp & 3) * 4;
+            lw[pp][0] = *reinterpret_cast<const uint2 *>(s0 + off + lane * 16 + wo);
+            lw[pp][1] = *reinterpret_cast<const uint2 *>(s1 + off + lane * 16 + wo);
+            kw[pp][0] = *reinterpret_cast<const uint2 *>(s0 + off + SOFF + g * 16 + wo);
+            kw[pp][1] = *reinterpret_cast<const uint2 *>(s1 + off + SOFF + g * 16 + wo);
+            if (kBits == 3) {
+                hw[pp][0] = *reinterpret_cast<const uint32_t *>(s0 + off + kLoBytes + lane * 8 + wo / 2);
+                hw[pp][1] = *reinterpret_cast<const uint32_t *>(s1 + off + kLoBytes + lane * 8 + wo / 2);
             }
-            const uint32_t s0 = comp4(sc0, blk), s1 = comp4(sc1, blk);
-            const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&s0));
-            const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&s1));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int pp = i >> 1, e = i & 1;
+            uint32_t bb0, bb1, bb2, bb3;
+            b_frag<kSrc>(rowp, (b + i) * 32, lane, bb0, bb1, bb2, bb3);
+            const float c0 = kMagic ? ca[b + i] : 0.0f, c1 = kMagic ? cb[b + i] : 0.0f;
+            float d0[4], d1[4];
+            block_dot<kBits, kMagic>(d0, e ? lw[pp][0].y : lw[pp][0].x,
+                                     kBits == 3 ? hw[pp][0] : 0u, 8 * e, bb0, bb1, bb2, bb3, c0,
+                                     c1);
+            block_dot<kBits, kMagic>(d1, e ? lw[pp][1].y : lw[pp][1].x,
+                                     kBits == 3 ? hw[pp][1] : 0u, 8 * e, bb0, bb1, bb2, bb3, c0,
+                                     c1);
+            const uint32_t w0 = e ? kw[pp][0].y : kw[pp][0].x;
+            const uint32_t w1 = e ? kw[pp][1].y : kw[pp][1].x;
+            const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+            const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
             acc0[0] = fmaf(f0.x, d0[0], acc0[0]);
             acc0[1] = fmaf(f0.x, d0[1], acc0[1]);
             acc0[2] = fmaf(f0.y, d0[2], acc0[2]);
@@ -194,6 +292,36 @@ STRATA_DEV void fused_slab2(float (&acc0)[4], float (&acc1)[4], const uint8_t *w
             acc1[3] = fmaf(f1.y, d1[3], acc1[3]);
         }
     }
+    // the last one to three blocks, one at a time
+    for (; b < b1; b++) {
+        const uint8_t *u0 = s0 + (b >> 2) * UB, *u1 = s1 + (b >> 2) * UB;
+        const int blk = b & 3;
+        const uint32_t lw0 = *reinterpret_cast<const uint32_t *>(u0 + lane * 16 + blk * 4);
+        const uint32_t lw1 = *reinterpret_cast<const uint32_t *>(u1 + lane * 16 + blk * 4);
+        const uint32_t kw0 = *reinterpret_cast<const uint32_t *>(u0 + SOFF + g * 16 + blk * 4);
+        const uint32_t kw1 = *reinterpret_cast<const uint32_t *>(u1 + SOFF + g * 16 + blk * 4);
+        uint32_t hw0 = 0, hw1 = 0;
+        if (kBits == 3) {
+            hw0 = *reinterpret_cast<const uint32_t *>(u0 + kLoBytes + lane * 8 + (blk >> 1) * 4);
+            hw1 = *reinterpret_cast<const uint32_t *>(u1 + kLoBytes + lane * 8 + (blk >> 1) * 4);
+        }
+        uint32_t bb0, bb1, bb2, bb3;
+        b_frag<kSrc>(rowp, b * 32, lane, bb0, bb1, bb2, bb3);
+        const float c0 = kMagic ? ca[b] : 0.0f, c1 = kMagic ? cb[b] : 0.0f;
+        float d0[4], d1[4];
+        block_dot<kBits, kMagic>(d0, lw0, hw0, 8 * (blk & 1), bb0, bb1, bb2, bb3, c0, c1);
+        block_dot<kBits, kMagic>(d1, lw1, hw1, 8 * (blk & 1), bb0, bb1, bb2, bb3, c0, c1);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&kw0));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&kw1));
+        acc0[0] = fmaf(f0.x, d0[0], acc0[0]);
+        acc0[1] = fmaf(f0.x, d0[1], acc0[1]);
+        acc0[2] = fmaf(f0.y, d0[2], acc0[2]);
+        acc0[3] = fmaf(f0.y, d0[3], acc0[3]);
+        acc1[0] = fmaf(f1.x, d1[0], acc1[0]);
+        acc1[1] = fmaf(f1.x, d1[1], acc1[1]);
+        acc1[2] = fmaf(f1.y, d1[2], acc1[2]);
+        acc1[3] = fmaf(f1.y, d1[3], acc1[3]);
+    }
 }
 
 // Bounded wait for an mbarrier phase by one thread; false (and the error
@@ -201,7 +329,7 @@ STRATA_DEV void fused_slab2(float (&acc0)[4], float (&acc1)[4], const uint8_t *w
 STRATA_DEV bool fwait(uint64_t *bar, uint32_t parity, const FusedParams &p,
                       volatile int *abort_flag) {
     long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 1000)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > p.budget) {
             atomicCAS(p.err, 0, kErrTimeout);
@@ -210,6 +338,14 @@ STRATA_DEV bool fwait(uint64_t *bar, uint32_t parity, const FusedParams &p,
         }
     }
     return true;
+}
+
+// The same wait for a whole warp: lane 0 waits, every lane gets its verdict.
+STRATA_DEV bool warp_fwait(uint64_t *bar, uint32_t parity, const FusedParams &p,
+                           volatile int *abort_flag, int lane) {
+    int ok = 0;
+    if (lane == 0) ok = fwait(bar, parity, p, abort_flag) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Bounded wait until a global counter reaches `target` (acquire).
@@ -226,30 +362,70 @@ STRATA_DEV bool fwait_count(const int *cnt, int target, const FusedParams &p,
             *abort_flag = 1;
             return false;
         }
-        __nanosleep(256);
+        __nanosleep(128);
     }
 }
 
-STRATA_DEV void group_sync(int group) {
-    asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory");
+// Grid barrier: arrive (release), then wait (acquire, bounded) until the
+// counter reaches `target`.
+STRATA_DEV bool grid_barrier(unsigned long long *bar, unsigned long long target,
+                             const FusedParams &p, volatile int *abort_flag) {
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(bar) : "memory");
+    long long t0 = clock64();
+    while (true) {
+        unsigned long long v;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(bar) : "memory");
+        if (v >= target) return true;
+        if (clock64() - t0 > p.budget) {
+            atomicCAS(p.err, 0, kErrTimeout);
+            *abort_flag = 1;
+            return false;
+        }
+        __nanosleep(32);
+    }
 }
 
-// misc ints: [1] abort flag, [2..34] scan scratch, [36 + g] and [88 + g]
-// group go/stop flags, [40 + 9 g] combine list of group g (count, then up to
-// 8 tokens), [80 + slot] item id of each ring slot
-constexpr int kMiscAbort = 1, kMiscScan = 2, kMiscFlag = 36, kMiscComb = 40, kMiscMeta = 80,
-              kMiscFlag2 = 88;
-constexpr int kItemEnd = -1;  // ring slot marker: no more items for this CTA
+// Smallest e >= 0 with v * 2^-e <= 2^7 (v >= 0), from the float's exponent.
+STRATA_DEV int prescale_exp(float v) {
+    const int b = (__float_as_int(v) >> 23) & 0xff;     // biased exponent
+    if (b == 0) return 0;                                // zero / subnormal
+    const int e = b - 127 + ((__float_as_int(v) & 0x7fffff) ? 1 : 0);  // ceil(log2 v)
+    return e > 7 ? e - 7 : 0;
+}
+STRATA_DEV float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
 
+// The expert token operand of column i of a token row, and the block
+// correction of the magic-offset form (2-bit): B_i = fp16(x_i 2^-ex s(i mod 32)),
+// corr = -sum over the block's 32 columns, in ascending order, of c(kk) B.
 template <int kBits>
+STRATA_DEV __half token_operand(float x, int ex, int i) {
+    const float v = x * pow2f(-ex);
+    return __float2half_rn(kBits == 2 ? v * magic_col_scale(i & 31) : v);
+}
+template <int kBits>
+STRATA_DEV float block_correction(const __nv_bfloat16 *blk, int ex) {
+    float v = 0.0f;
+#pragma unroll 8
+    for (int kk = 0; kk < 32; kk++)
+        v = fmaf(-magic_col_corr(kk),
+                 __half2float(token_operand<kBits>(__bfloat162float(blk[kk]), ex, kk)), v);
+    return v;
+}
+
+template <int kBits, bool kStaged>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedParams p) {
-    extern __shared__ __align__(16) uint8_t sm[];
+    extern __shared__ __align__(128) uint8_t sm[];
     constexpr int UB = unit_bytes(kBits);
-    const FusedSmem L =
-        fused_smem(p.T, p.E, p.k, p.H, p.Ip, p.ring, p.item_bytes, p.staged, p.units_max);
+    constexpr bool kMagic = kBits == 2;
+    const FusedSmem L = fused_smem(p.T, p.E, p.k, p.H, p.Ip, p.ring, p.item_bytes, p.staged,
+                                   p.units_max, p.na);
     uint8_t *ring = sm + L.ring;
-    __half *xs = reinterpret_cast<__half *>(sm + L.xs);
     float *red = reinterpret_cast<float *>(sm + L.red);
+    uint2 *xi = reinterpret_cast<uint2 *>(sm + L.red);  // while routing
+    __half *xs = reinterpret_cast<__half *>(sm + L.xs);
+    float *scorr = reinterpret_cast<float *>(sm + L.corr);  // [T][H / 32]
+    __nv_bfloat16 *xb = reinterpret_cast<__nv_bfloat16 *>(sm + L.rega);
+    __half *abuf0 = reinterpret_cast<__half *>(sm + L.rega);
     int *sidx = reinterpret_cast<int *>(sm + L.sidx);
     float *sw = reinterpret_cast<float *>(sm + L.sw);
     int *sslot = reinterpret_cast<int *>(sm + L.sslot);
@@ -258,293 +434,800 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     int *soff = reinterpret_cast<int *>(sm + L.soff);
     int4 *units = reinterpret_cast<int4 *>(sm + L.units);
     int *slist = reinterpret_cast<int *>(sm + L.slist);
+    int *sex = reinterpret_cast<int *>(sm + L.sex);
     int *misc = reinterpret_cast<int *>(sm + L.misc);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + L.bars);
     uint64_t *empty = full + kFMaxRing;
     uint64_t *xbar = empty + kFMaxRing;
-    uint64_t *abar = xbar + 2;  // [kFGroups]
+    uint64_t *lgbar = xbar + 1, *rdy = xbar + 2, *pickbar = xbar + 3, *rdy2 = xbar + 4,
+             *dsp = xbar + 5;
+    uint64_t *abar = xbar + 8;       // [kMaxA] activation rows landed
+    uint64_t *aempty = abar + kMaxA; // [kMaxA] the group's warps are done with them
     volatile int *abort_flag = misc + kMiscAbort;
+    volatile int *vmisc = misc;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x, cta = blockIdx.x;
     const int T = p.T, E = p.E, k = p.k, H = p.H, Tk = T * k;
+    const int ns4 = H / 128, nbh = H / 32, nbi = p.Ip / 32;
+    const int nsl = p.Ip / kSlabRows;              // gate/up slabs per unit
+    const int ndn = H / (kSlabRows * kDownSlabs);  // down blocks per unit
+    const int nsh = (T + kFTile - 1) / kFTile;     // shared-expert units
+    constexpr bool staged = kStaged;  // token rows in shared memory (T <= 8)
+    const int e0 = (int)((long long)cta * E / G), e1 = (int)((long long)(cta + 1) * E / G);
+    const int ne = e1 - e0;
+    const int wbytes = ne * H * 4;                                 // router slice
+    const int nwc = (wbytes + p.item_bytes - 1) / p.item_bytes;    // ring positions it takes
+    const int nxs = staged ? nsh * nsl : 0;                        // extras over the grid
+    const int nx = cta < nxs ? (nxs - 1 - cta) / G + 1 : 0;        // this CTA's extras
+    const size_t gu_bytes = (size_t)p.nseg_h * UB, dn_bytes = (size_t)kDownSlabs * p.nseg_i * UB;
+
+    for (int i = tid; i < 256; i += blockDim.x) misc[i] = 0;
+    __syncthreads();
     if (tid == 0) {
         for (int s = 0; s < p.ring; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], kGWarps);  // the warps of the group
         }
         mbar_init(xbar, 1);
-        for (int i = 0; i < kFGroups; i++) mbar_init(&abar[i], 1);
-        misc[kMiscAbort] = 0;
+        mbar_init(lgbar, kFWarps);
+        mbar_init(rdy, 1);
+        mbar_init(pickbar, 1);
+        mbar_init(rdy2, 1);
+        mbar_init(dsp, 1);
+        for (int b = 0; b < p.na; b++) {
+            mbar_init(&abar[b], 1);
+            mbar_init(&aempty[b], kGWarps);
+        }
         fence_mbar_init();
     }
-    for (int e = tid; e < E; e += blockDim.x) mask[e] = 0ull;
-    // everything below reads what the router wrote
-    grid_dependency_wait();
     __syncthreads();
 
-    // ------------------------------------------------------------- dispatch
-    for (int i = tid; i < Tk; i += blockDim.x) {
-        sidx[i] = __ldcg(p.idx + i);
-        sw[i] = __ldcg(p.wts + i);
-    }
-    __syncthreads();
-    for (int i = tid; i < Tk; i += blockDim.x) atomicOr(&mask[sidx[i]], 1ull << (i / k));
-    __syncthreads();
-    // one scan of (count << 16 | units): both sums stay below 2^16 (T k <= 1024)
-    // thread tid owns experts [tid ept, tid ept + ept) (E <= 2 blockDim.x)
-    const int ept = (E + blockDim.x - 1) / blockDim.x, eb = tid * ept;
-    int local = 0;
-    for (int e = eb; e < eb + ept && e < E; e++) {
-        const int c = __popcll(mask[e]);
-        local += (c << 16) | ((c + kFTile - 1) / kFTile);
-    }
-    int packed_total;
-    int packed = cta_exclusive_scan(local, misc + kMiscScan, &packed_total);
-    const int utot = packed_total & 0xffff;
-    const int nsh = (T + kFTile - 1) / kFTile;
-    for (int e = eb; e < eb + ept && e < E; e++) {
-        const int c = __popcll(mask[e]), nu = (c + kFTile - 1) / kFTile;
-        const int off = packed >> 16, us = packed & 0xffff;
-        soff[e] = off;
-        for (int i = 0; i < nu; i++) {
-            const int n = c - i * kFTile;
-            units[nsh + us + i] = make_int4(e, off + i * kFTile, n < kFTile ? n : kFTile, 0);
+    // the routed item list, once dispatch has run (same in every role)
+    auto item_counts = [&](int &Ng, int &N2, int &ug0) {
+        const int n_units = vmisc[kMiscNUnits];
+        ug0 = staged ? nsh : 0;  // with extras, the shared units' slabs are done already
+        Ng = (n_units - ug0) * nsl;
+        N2 = n_units * ndn;
+    };
+
+    // =========================================================== copy warp
+    if (warp == kWCopy) {
+        if (lane != 0) return;
+        const uint64_t pol = l2_evict_first_policy();  // weights: read once per forward
+        int pos = 0;
+        bool ok = true;
+        auto acquire = [&](int ps) {  // wait until ring position ps may be filled
+            return ps < p.ring || fwait(&empty[ps % p.ring], ((ps / p.ring) - 1) & 1, p, abort_flag);
+        };
+        auto issue_gu = [&](int slot, int e, int slab) {
+            const uint8_t *wg = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
+                                (size_t)slab * gu_bytes;
+            uint8_t *dst = ring + (size_t)slot * p.item_bytes;
+            mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * gu_bytes));
+            bulk_g2s_hint(dst, wg, (uint32_t)gu_bytes, &full[slot], pol);
+            bulk_g2s_hint(dst + gu_bytes, wg + p.mat_bytes, (uint32_t)gu_bytes, &full[slot], pol);
+        };
+        // router slice: constant, requested before the previous kernel ends
+        const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(p.Wp) + (size_t)e0 * H * 4;
+        for (int i = 0; i < nwc; i++, pos++) {
+            const int bytes = wbytes - i * p.item_bytes < p.item_bytes ? wbytes - i * p.item_bytes
+                                                                       : p.item_bytes;
+            mbar_arrive_expect_tx(&full[pos], (uint32_t)bytes);
+            bulk_g2s_hint(ring + (size_t)pos * p.item_bytes, wsrc + (size_t)i * p.item_bytes,
+                          (uint32_t)bytes, &full[pos], pol);
         }
-        packed += (c << 16) | nu;
-    }
-    if (tid < nsh) {
-        const int n = T - tid * kFTile;
-        units[tid] = make_int4(E, Tk + tid * kFTile, n < kFTile ? n : kFTile, 0);
-    }
-    __syncthreads();
-    for (int i = tid; i < Tk; i += blockDim.x) {
-        const int t = i / k, ej = sidx[i];
-        const int pos = soff[ej] + __popcll(mask[ej] & ((1ull << t) - 1ull));
-        slist[pos] = t;
-        sslot[i] = pos;
-        int rank = 0;
-        for (int jj = 0; jj < k; jj++) rank += sidx[t * k + jj] < ej;
-        sord[t * k + rank] = i;  // combine order: ascending expert id
-    }
-    __syncthreads();
-
-    // --------------------------------------------------------------- items
-    const int n_units = nsh + utot;
-    const int nsl = p.Ip / kSlabRows;                 // gate/up items per unit
-    const int ndn = H / (kSlabRows * kDownSlabs);     // down items per unit
-    const int N1 = n_units * nsl, N2 = n_units * ndn;
-    // items are claimed from two global queues (gate/up first, then down):
-    // a CTA that finishes early takes more, so the last CTA does not trail
-    const bool staged = p.staged != 0;
-    int *meta = misc + kMiscMeta;  // item id of each ring slot (or kItemEnd)
-    const size_t gu_bytes = (size_t)p.nseg_h * UB, dn_bytes = (size_t)kDownSlabs * p.nseg_i * UB;
-
-    if (warp == kFWarps) {
-        // ---------------------------------------------------- copy warp
-        if (lane == 0) {
-            if (staged) {
-                mbar_arrive_expect_tx(xbar, (uint32_t)(T * H * 2));
-                for (int t = 0; t < T; t++)
-                    bulk_g2s(xs + (size_t)t * (H + 8), p.x16 + (size_t)t * H, (uint32_t)(H * 2),
-                             xbar);
-            }
-            // claim items until both queues are empty, then leave one end
-            // marker per group (a marker completes its slot with no bytes)
-            int j = 0, ended = 0;
-            bool gu_left = true, dn_left = true;
-            for (; ended < kFGroups; j++) {
-                const int slot = j % p.ring;
-                if (j >= p.ring && !fwait(&empty[slot], ((j / p.ring) - 1) & 1, p, abort_flag))
-                    break;
-                int item = kItemEnd;
-                if (gu_left) {
-                    const int gq = atomicAdd(p.queue, 1);
-                    if (gq < N1) item = gq;
-                    else gu_left = false;
-                }
-                if (item == kItemEnd && dn_left) {
-                    const int dq = atomicAdd(p.queue + 1, 1);
-                    if (dq < N2) item = N1 + dq;
-                    else dn_left = false;
-                }
-                meta[slot] = item;  // published by the arrive below
-                uint8_t *dst = ring + (size_t)slot * p.item_bytes;
-                if (item == kItemEnd) {
-                    mbar_arrive(&full[slot]);
-                    ended++;
-                } else if (item < N1) {
-                    const int u = item / nsl, slab = item % nsl;
-                    const int e = units[u].x;
-                    const uint8_t *wg = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
-                                        (size_t)slab * gu_bytes;
-                    mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * gu_bytes));
-                    const uint64_t pol = l2_evict_first_policy();  // weights: read once
-                    bulk_g2s_hint(dst, wg, (uint32_t)gu_bytes, &full[slot], pol);
-                    bulk_g2s_hint(dst + gu_bytes, wg + p.mat_bytes, (uint32_t)gu_bytes, &full[slot],
-                                  pol);
+        grid_dependency_wait();  // the token rows are the previous kernel's output
+        if (staged) {
+            mbar_arrive_expect_tx(xbar, (uint32_t)(T * H * 2));
+            for (int t = 0; t < T; t++)
+                bulk_g2s(xb + (size_t)t * H, p.x + (size_t)t * H, (uint32_t)(H * 2), xbar);
+        }
+        // the shared expert's gate/up slabs of this CTA (no routing needed)
+        int mx = 0;
+        for (; mx < nx && ok; mx++) {
+            const int ps = pos + mx, slot = ps % p.ring, i = cta + mx * G;
+            ok = acquire(ps);
+            if (!ok) break;
+            vmisc[kMiscMeta + slot] = (kKindExtra << 28) | i;
+            issue_gu(slot, E, i % nsl);
+        }
+        pos += mx;  // positions issued so far
+        if (ok) ok = fwait(dsp, 0, p, abort_flag);
+        if (ok) {
+            int Ng, N2, ug0;
+            item_counts(Ng, N2, ug0);
+            const int W = Ng + N2;
+            int kd = 0;
+            for (int it = cta; it < W && ok; it += G, pos++) {
+                ok = acquire(pos);
+                if (!ok) break;
+                const int slot = pos % p.ring;
+                if (it < Ng) {
+                    const int u = ug0 + it / nsl;
+                    vmisc[kMiscMeta + slot] = (kKindGU << 28) | it;
+                    issue_gu(slot, units[u].x, it % nsl);
                 } else {
-                    const int di = item - N1, u = di / ndn, rg = di % ndn;
-                    const int e = units[u].x;
+                    const int d = it - Ng, u = d / ndn, e = units[u].x;
+                    vmisc[kMiscMeta + slot] = (kKindDown << 28) | (kd << 20) | d;
+                    kd++;
                     const uint8_t *wd = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
-                                        2 * p.mat_bytes + (size_t)rg * dn_bytes;
+                                        2 * p.mat_bytes + (size_t)(d % ndn) * dn_bytes;
                     mbar_arrive_expect_tx(&full[slot], (uint32_t)dn_bytes);
-                    bulk_g2s_hint(dst, wd, (uint32_t)dn_bytes, &full[slot],
-                                  l2_evict_first_policy());
+                    bulk_g2s_hint(ring + (size_t)slot * p.item_bytes, wd, (uint32_t)dn_bytes,
+                                  &full[slot], pol);
                 }
             }
-            // the CTA must not exit with copies in flight (abort path)
-            for (int i = j > p.ring ? j - p.ring : 0; i < j; i++)
-                mbar_drain(&full[i % p.ring], (i / p.ring) & 1);
-            if (staged) mbar_drain(xbar, 0);
+            // one end marker per group (completes its slot without bytes)
+            for (int gq = 0; gq < kGroups && ok; gq++) {
+                ok = acquire(pos);
+                if (!ok) break;
+                vmisc[kMiscMeta + pos % p.ring] = kItemEnd;
+                mbar_arrive(&full[pos % p.ring]);
+                pos++;
+            }
+        }
+        // the CTA must not exit with copies in flight (abort path)
+        for (int i = pos > p.ring ? pos - p.ring : 0; i < pos; i++)
+            mbar_drain(&full[i % p.ring], (i / p.ring) & 1);
+        if (staged) mbar_drain(xbar, 0);
+        return;
+    }
+
+    // ====================================================== publish warp
+    // Finished gate/up slabs -> per-unit counts: the warp that completes a
+    // slab posts its unit in a shared-memory queue (CTA scope); this warp makes
+    // each batch visible at gpu scope with one fence and then counts it.
+    if (warp == kWPub) {
+        if (lane != 0) return;
+        grid_dependency_wait();
+        unsigned long long b0;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
+        const int par = (int)((b0 / (2ull * (unsigned long long)G)) & 1ull);
+        int *done_gu = p.cnt + (size_t)par * p.cnt_stride;
+        int seen = 0;
+        long long t_idle = clock64();
+        while (!*abort_flag) {
+            const int done = vmisc[kMiscWarpsDone];
+            __threadfence_block();
+            int n = 0;
+            while (n < kPubQ && vmisc[kMiscPubQ + (seen + n) % kPubQ] != 0) n++;
+            if (n > 0) {
+                __threadfence_block();
+                asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                for (int i = 0; i < n; i++) {
+                    const int s = kMiscPubQ + (seen + i) % kPubQ;
+                    asm volatile("red.relaxed.gpu.global.add.s32 [%0], 1;" ::"l"(
+                                     done_gu + vmisc[s] - 1)
+                                 : "memory");
+                    vmisc[s] = 0;
+                }
+                seen += n;
+                __threadfence_block();
+                vmisc[kMiscPubSeen] = seen;
+                t_idle = clock64();
+            } else {
+                if (done == kFWarps && vmisc[kMiscPubN] == seen) break;  // all posted and counted
+                if (clock64() - t_idle > p.budget) {
+                    atomicCAS(p.err, 0, kErrTimeout);
+                    *abort_flag = 1;
+                    break;
+                }
+                __nanosleep(200);
+            }
         }
         return;
     }
 
-    // ------------------------------------------------------ compute groups
-    const int gi = warp >> 2, q = warp & 3, gtid = tid & 127;
-    const int sa = q * p.nseg_h / 4, sb = (q + 1) * p.nseg_h / 4;
-    const int g = lane >> 2, cq = lane & 3;
-    const int per_blk = k + 1;  // down items that write one (token, row block)
-    int *flag = misc + kMiscFlag + gi;
-    int *flag2 = misc + kMiscFlag2 + gi;  // second go/stop word of a down item
-    int *comb = misc + kMiscComb + 9 * gi;
-    __half *abuf = reinterpret_cast<__half *>(sm + L.abuf) + (size_t)gi * kFTile * (p.Ip + 8);
-    uint32_t a_uses = 0;  // phases of abar[gi] used so far (thread gtid 0)
-    if (staged) {
-        // one waiter per group, the answer shared through the group barrier
-        if (gtid == 0) *flag = fwait(xbar, 0, p, abort_flag) ? 1 : 0;
-        group_sync(gi);
-        if (!*flag) return;
-        group_sync(gi);
-    }
-    for (int j = gi;; j += kFGroups) {
-        const int slot = j % p.ring;
-        if (gtid == 0) *flag = fwait(&full[slot], (j / p.ring) & 1, p, abort_flag) ? 1 : 0;
-        group_sync(gi);
-        if (!*flag) return;  // the whole group leaves together
-        const int item = meta[slot];
-        if (item == kItemEnd) break;
-        const bool is_gu = item < N1;
-        const int u = is_gu ? item / nsl : (item - N1) / ndn;
-        const int part = is_gu ? item % nsl : (item - N1) % ndn;
-        const int4 un = units[u];
-        const int slot0 = un.y, n = un.z;
-        if (!is_gu) {
-            // a down item needs every gate/up slab of its unit (other CTAs);
-            // then its n activation rows come in with one bulk copy each
-            if (gtid == 0) {
-                bool ok = fwait_count(p.done_gu + u, nsl, p, abort_flag);
-                if (ok) {
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    mbar_arrive_expect_tx(&abar[gi], (uint32_t)(n * p.Ip * 2));
-                    for (int r = 0; r < n; r++)
-                        bulk_g2s(abuf + (size_t)r * (p.Ip + 8), p.a + (size_t)(slot0 + r) * p.Ip,
-                                 (uint32_t)(p.Ip * 2), &abar[gi]);
-                    ok = fwait(&abar[gi], a_uses & 1, p, abort_flag);
-                    if (!ok) mbar_drain(&abar[gi], a_uses & 1);
-                    a_uses++;
-                }
-                *flag2 = ok ? 1 : 0;
-            }
-            group_sync(gi);
-            if (!*flag2) return;
+    // ======================================================== fetch warp
+    // Grid barrier(s), then the activation rows of this CTA's down blocks.
+    if (warp == kWFetch) {
+        grid_dependency_wait();
+        {
+            // run the top-k code once on stale logits while the router works, so
+            // its instructions are in this SM's caches when the routing needs them
+            int pe;
+            float pw;
+            warp_topk(p.logits, E, k, lane, pe, pw);
+            if (pe == 0x7fffffff && pw == 1.0f) misc[kMiscTmp] = 1;  // keeps the call
         }
-        const uint8_t *w = ring + (size_t)slot * p.item_bytes;
-        if (is_gu) {
-            // ------------------------------------------------ gate/up item
-            float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
-            if (staged) {
-                const int r = lane & 7, sl = slot0 + (r < n ? r : 0);
-                const __half *rowp = xs + (size_t)(sl < Tk ? slist[sl] : sl - Tk) * (H + 8);
-                fused_slab2<kBits, kSrcSmem>(accg, accu, w + sa * UB, w + gu_bytes + sa * UB,
-                                             sb - sa, rowp, sa * 128, lane);
-            } else {
-                const int sl = slot0 + (g < n ? g : 0);
-                const __half *rowp = p.x16 + (size_t)(sl < Tk ? slist[sl] : sl - Tk) * H;
-                fused_slab2<kBits, kSrcLdg>(accg, accu, w + sa * UB, w + gu_bytes + sa * UB,
-                                            sb - sa, rowp, sa * 128, lane);
+        if (lane != 0) return;
+        unsigned long long b0;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
+        const unsigned long long gg = (unsigned long long)G, ep = b0 / (2ull * gg);
+        const int par = (int)(ep & 1ull);
+        int *done_gu = p.cnt + (size_t)par * p.cnt_stride;
+        // the other counter set is the next launch's: zero this CTA's share
+        int *other = p.cnt + (size_t)(1 - par) * p.cnt_stride;
+        for (int i = (int)((long long)cta * p.cnt_stride / G);
+             i < (int)((long long)(cta + 1) * p.cnt_stride / G); i++)
+            other[i] = 0;
+        bool ok = fwait(lgbar, 0, p, abort_flag);  // this CTA's logits are stored
+        // every CTA arrives, also after a failed wait, so the count stays whole
+        ok = grid_barrier(p.bar, 2ull * gg * ep + gg, p, abort_flag) && ok;
+        if (ok) mbar_arrive(rdy);
+        if (T > kTopkLocalT) {
+            if (ok) ok = fwait(pickbar, 0, p, abort_flag);
+            ok = grid_barrier(p.bar, 2ull * gg * (ep + 1), p, abort_flag) && ok;
+            if (ok) mbar_arrive(rdy2);
+        } else {
+            asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(p.bar) : "memory");
+        }
+        if (ok) ok = fwait(dsp, 0, p, abort_flag);
+        int issued = 0;
+        if (ok) {
+            int Ng, N2, ug0;
+            item_counts(Ng, N2, ug0);
+            const int W = Ng + N2;
+            int first = cta;
+            if (first < Ng) first += ((Ng - first + G - 1) / G) * G;  // first down position
+            for (int it = first; it < W && ok; it += G, issued++) {
+                const int d = it - Ng, u = d / ndn, kd = issued, b = kd % p.na;
+                const int4 un = units[u];
+                // buffer b is free once the group's warps are done with its last block
+                if (kd >= p.na && !(ok = fwait(&aempty[b], ((kd / p.na) - 1) & 1, p, abort_flag)))
+                    break;
+                ok = fwait_count(done_gu + u, nsl, p, abort_flag);
+                if (!ok) break;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __half *dst = abuf0 + (size_t)b * kFTile * (p.Ip + 8);
+                mbar_arrive_expect_tx(&abar[b], (uint32_t)(un.z * p.Ip * 2));
+                for (int r = 0; r < un.z; r++)
+                    bulk_g2s(dst + (size_t)r * (p.Ip + 8), p.a + (size_t)(un.y + r) * p.Ip,
+                             (uint32_t)(p.Ip * 2), &abar[b]);
             }
-            float *rd = red + ((gi * 4 + q) * 32 + lane) * 8;
+        }
+        // no exit with copies in flight
+        for (int i = issued > p.na ? issued - p.na : 0; i < issued; i++)
+            mbar_drain(&abar[i % p.na], (i / p.na) & 1);
+        return;
+    }
+
+    // ====================================================== combine warp
+    // Finished down blocks: count every token's finished (token, 128-row
+    // block) pairs (one gpu-scope fence per batch) and combine each pair that
+    // is complete: y = Y_shared + sum over the picks in ascending expert id of
+    // w Y, in fp32, the token's prescale off, one rounding to bf16 (with the
+    // residual added in the stack).
+    if (warp == kWComb) {
+        grid_dependency_wait();
+        unsigned long long b0;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
+        const int par = (int)((b0 / (2ull * (unsigned long long)G)) & 1ull);
+        int *done_tok = p.cnt + (size_t)par * p.cnt_stride + p.cnt_tok;
+        const int per_blk = k + 1;  // down blocks that write one (token, row block)
+        int seen = 0;
+        long long t_idle = clock64();
+        while (true) {
+            int n = 0, fin = 0, stop = 0;
+            if (lane == 0) {
+                stop = *abort_flag;
+                fin = vmisc[kMiscWarpsDone] == kFWarps;
+                __threadfence_block();
+                while (n < kPubQ && vmisc[kMiscCombQ + (seen + n) % kPubQ] != 0) n++;
+                if (n == 0 && fin && vmisc[kMiscCombN] != seen) fin = 0;
+            }
+            n = __shfl_sync(0xffffffffu, n, 0);
+            fin = __shfl_sync(0xffffffffu, fin, 0);
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop) break;
+            if (n == 0) {
+                if (fin) break;  // every block is posted and combined
+                int late = 0;
+                if (lane == 0 && clock64() - t_idle > p.budget) {
+                    atomicCAS(p.err, 0, kErrTimeout);
+                    *abort_flag = 1;
+                    late = 1;
+                }
+                if (__shfl_sync(0xffffffffu, late, 0)) break;
+                __nanosleep(500);
+                continue;
+            }
+            __syncwarp();
+            __threadfence();  // the posted blocks' rows, at gpu scope, before the counts
+            for (int i = 0; i < n; i++) {
+                const int v = vmisc[kMiscCombQ + (seen + i) % kPubQ] - 1;
+                const int u = v / ndn, part = v % ndn;
+                const int4 un = units[u];
+                int t = 0, c = 0;
+                if (lane < un.z) {
+                    const int sl = un.y + lane;
+                    t = sl < Tk ? slist[sl] : sl - Tk;
+                    c = atomicAdd(done_tok + t * ndn + part, 1);
+                }
+                unsigned ready = __ballot_sync(0xffffffffu, lane < un.z && c == per_blk - 1);
+                if (ready) __threadfence();  // the other blocks' rows of these tokens
+                while (ready) {
+                    const int j = __ffs(ready) - 1;
+                    ready &= ready - 1;
+                    const int tt = __shfl_sync(0xffffffffu, t, j);
+                    const int ex = staged ? sex[tt] : __ldcg(p.xex + tt);
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                rd[i] = accg[i];
-                rd[4 + i] = accu[i];
+                    for (int cc = 0; cc < 4; cc++) {
+                        const int col = part * kSlabRows * kDownSlabs + cc * 32 + lane;
+                        float vv[kFMaxK];
+#pragma unroll
+                        for (int r = 0; r < kFMaxK; r++)
+                            vv[r] = r < k ? __ldcg(p.Y + (size_t)sslot[sord[tt * k + r]] * H + col)
+                                          : 0.0f;
+                        float acc2 = __ldcg(p.Y + (size_t)(Tk + tt) * H + col);
+#pragma unroll
+                        for (int r = 0; r < kFMaxK; r++)
+                            if (r < k) acc2 = fmaf(sw[sord[tt * k + r]], vv[r], acc2);
+                        if (ex) acc2 *= pow2f(2 * ex);
+                        __nv_bfloat16 *o = p.out + (size_t)tt * H + col;
+                        const __nv_bfloat16 yb = __float2bfloat16_rn(acc2);
+                        *o = p.residual ? __float2bfloat16_rn(__fadd_rn(__bfloat162float(*o),
+                                                                        __bfloat162float(yb)))
+                                        : yb;
+                    }
+                }
             }
-            group_sync(gi);
-            if (gtid == 0) mbar_arrive(&empty[slot]);  // the weights are consumed
-            if (q == 0) {
-                const float *r0 = red + ((gi * 4 + 0) * 32 + lane) * 8;
-                const float *r1 = r0 + 32 * 8, *r2 = r1 + 32 * 8, *r3 = r2 + 32 * 8;
+            __syncwarp();
+            if (lane == 0) {
+                for (int i = 0; i < n; i++) vmisc[kMiscCombQ + (seen + i) % kPubQ] = 0;
+                __threadfence_block();
+                vmisc[kMiscCombSeen] = seen + n;
+            }
+            seen += n;
+            t_idle = clock64();
+        }
+        return;
+    }
+
+    // ==================================================== compute warps
+    const int g = lane >> 2, cq = lane & 3;
+    // compute-wide verdicts go through one slot, written by thread 0 before a
+    // compute barrier and read by every compute thread after it
+    volatile int *cflag = misc + kMiscCFlag;
+    grid_dependency_wait();
+    if (tid == 0) {
+        unsigned long long b0;
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
+        misc[kMiscPar] = (int)((b0 / (2ull * (unsigned long long)G)) & 1ull);
+    }
+    for (int e = tid; e < E; e += kFCompute) mask[e] = 0ull;  // dispatch, later
+    bool alive = true;
+
+    // ---- token rows.  Staged (T <= 8): the raw rows arrive by bulk copy; one
+    // pass builds the lane-interleaved bf16 copy the router reads (slot
+    // (t, s, l) holds x[t][128 s + 32 j + l], j = 0..3) while warps t < T sum
+    // the squares of row t in a fixed order for the token's prescale.
+    if (staged) {
+        if (tid == 0) *cflag = fwait(xbar, 0, p, abort_flag) ? 1 : 0;
+        compute_sync();
+        alive = *cflag != 0;
+        if (alive) {
+            const unsigned short *xu = reinterpret_cast<const unsigned short *>(xb);
+            for (int i = tid; i < T * ns4 * 32; i += kFCompute) {
+                const int t = i / (ns4 * 32), r = i % (ns4 * 32);
+                const unsigned short *px = xu + (size_t)t * H + (r >> 5) * 128 + (r & 31);
+                xi[i] = make_uint2((uint32_t)px[0] | ((uint32_t)px[32] << 16),
+                                   (uint32_t)px[64] | ((uint32_t)px[96] << 16));
+            }
+            if (warp < T) {
+                float ss = 0.0f;
+                for (int i = lane; i < H; i += 32) {
+                    const float v = __bfloat162float(xb[(size_t)warp * H + i]);
+                    ss = fmaf(v, v, ss);
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (lane == 0) sex[warp] = p.w2 > 0.0f ? prescale_exp(sqrtf(ss) * p.w2 * 1.001f) : 0;
+            }
+            compute_sync();
+        }
+    } else {
+        // this CTA writes the expert operand of tokens cta, cta + G, ... for every CTA
+        for (int t = cta; t < T; t += G) {
+            float ss = 0.0f;
+            for (int i = tid; i < H; i += kFCompute) {
+                const float v = __bfloat162float(p.x[(size_t)t * H + i]);
+                ss = fmaf(v, v, ss);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            float *rs = red;
+            if (lane == 0) rs[warp] = ss;
+            compute_sync();
+            if (tid == 0) {
+                float s = 0.0f;
+                for (int w = 0; w < kFWarps; w++) s += rs[w];
+                const int ex = p.w2 > 0.0f ? prescale_exp(sqrtf(s) * p.w2 * 1.001f) : 0;
+                misc[kMiscTmp] = ex;
+                p.xex[t] = ex;
+            }
+            compute_sync();
+            const int ex = misc[kMiscTmp];
+            for (int i = tid; i < H; i += kFCompute)
+                p.x16[(size_t)t * H + i] =
+                    token_operand<kBits>(__bfloat162float(p.x[(size_t)t * H + i]), ex, i);
+            if (kMagic)
+                for (int b = tid; b < nbh; b += kFCompute)
+                    p.corr[(size_t)t * nbh + b] = block_correction<kBits>(p.x + (size_t)t * H + 32 * b, ex);
+            compute_sync();
+        }
+    }
+
+    // ---- router logits of this CTA's experts (fixed summation order)
+    if (alive && nwc > 0) {
+        if (tid == 0) {
+            bool ok = true;
+            for (int s = 0; s < nwc && ok; s++) ok = fwait(&full[s], 0, p, abort_flag);
+            *cflag = ok ? 1 : 0;
+        }
+        compute_sync();
+        alive = *cflag != 0;
+    }
+    if (alive && ne > 0) {
+        const float4 *Ws = reinterpret_cast<const float4 *>(ring);  // [ne][H/128][32]
+        // staged rows: one (token, expert) task per warp; global rows: one
+        // token per warp, every expert of the CTA (each row read once)
+        const int per = staged ? 1 : ne;
+        const int ntask = staged ? T * ne : T;
+        for (int task = warp; task < ntask; task += kFWarps) {
+            const int t = staged ? task / ne : task;
+            const int eb = staged ? task % ne : 0;
+            for (int ee = eb; ee < eb + per; ee += 4) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int s0 = 0; s0 < ns4; s0 += 4) {
+                    float xv[4][4];
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        const int s4 = s0 + c;
+                        if (staged) {
+                            const uint2 v = s4 < ns4 ? xi[((size_t)t * ns4 + s4) * 32 + lane]
+                                                     : make_uint2(0u, 0u);
+                            xv[c][0] = __uint_as_float(v.x << 16);
+                            xv[c][1] = __uint_as_float(v.x & 0xffff0000u);
+                            xv[c][2] = __uint_as_float(v.y << 16);
+                            xv[c][3] = __uint_as_float(v.y & 0xffff0000u);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; j++)
+                                xv[c][j] = s4 < ns4 ? __bfloat162float(p.x[(size_t)t * H + 128 * s4 +
+                                                                           32 * j + lane])
+                                                    : 0.0f;
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; c++) {
+                        if (s0 + c >= ns4) break;
+#pragma unroll
+                        for (int b = 0; b < 4; b++) {
+                            if (ee + b >= eb + per) break;
+                            const float4 w = Ws[((size_t)(ee + b) * ns4 + s0 + c) * 32 + lane];
+                            acc[b] = fmaf(xv[c][0], w.x, acc[b]);
+                            acc[b] = fmaf(xv[c][1], w.y, acc[b]);
+                            acc[b] = fmaf(xv[c][2], w.z, acc[b]);
+                            acc[b] = fmaf(xv[c][3], w.w, acc[b]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                    if (ee + b >= eb + per) break;
+                    float v = acc[b];
+#pragma unroll
+                    for (int s = 16; s >= 1; s >>= 1)
+                        v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, s));
+                    if (lane == 0) {
+                        const int e = e0 + ee + b;
+                        p.logits[(size_t)t * E + e] = p.bias ? __fadd_rn(v, p.bias[e]) : v;
+                    }
+                }
+            }
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(lgbar);  // this warp's logits (and token rows) are stored
+    // the expert operand of the staged tokens and (2-bit) its block corrections
+    if (alive && staged) {
+        for (int i = tid; i < T * (H / 2); i += kFCompute) {
+            const int t = i / (H / 2), c = 2 * (i % (H / 2));
+            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(xb + (size_t)t * H + c);
+            __half2 h;
+            h.x = token_operand<kBits>(__bfloat162float(v.x), sex[t], c);
+            h.y = token_operand<kBits>(__bfloat162float(v.y), sex[t], c + 1);
+            *reinterpret_cast<__half2 *>(xs + (size_t)t * (H + 8) + c) = h;
+        }
+        if (kMagic)
+            for (int task = tid; task < T * nbh; task += kFCompute) {
+                const int t = task / nbh, b = task % nbh;
+                scorr[t * nbh + b] = block_correction<kBits>(xb + (size_t)t * H + 32 * b, sex[t]);
+            }
+    }
+    compute_sync();
+    if (tid == 0)
+        for (int s = 0; s < nwc; s++) mbar_arrive_cnt(&empty[s], kGWarps);  // router slice consumed
+
+    // ---- ring items: group gi (warps 8 gi .. 8 gi + 7) takes positions
+    // nwc + gi, nwc + gi + 2, ...; each of its warps takes a share of the item
+    //   gate/up slab: warp q an eighth of K of both the gate and the up slab;
+    //   down block: warp q the slabs 2 (q >> 1), 2 (q >> 1) + 1, half of K;
+    // and the last of the 8 to finish an item completes it.
+    const int gi = warp / kGWarps, q = warp % kGWarps;
+    int jpos = nwc + gi;
+    auto slot_exp = [&](int sl) -> int {  // the prescale exponent of a slot's token
+        const int t = sl < Tk ? slist[sl] : sl - Tk;
+        return staged ? sex[t] : __ldcg(p.xex + t);
+    };
+    auto slot_tok = [&](int sl) -> int { return sl < Tk ? slist[sl] : sl - Tk; };
+    // count this warp in for the item in `slot`; true for the last of the group
+    auto last_warp = [&](int slot) -> bool {
+        int old = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            old = atomicAdd(misc + kMiscGCnt + slot, 1);
+            if (old == kGWarps - 1) {
+                misc[kMiscGCnt + slot] = 0;  // before the slot can be refilled
+                __threadfence_block();
+            }
+        }
+        const bool last = __shfl_sync(0xffffffffu, old, 0) == kGWarps - 1;
+        __syncwarp();
+        return last;
+    };
+    auto run_items = [&](int stop) -> bool {  // false: aborted or end marker seen
+        for (; jpos < stop; jpos += kGroups) {
+            const int slot = jpos % p.ring;
+            if (!warp_fwait(&full[slot], (jpos / p.ring) & 1, p, abort_flag, lane)) return false;
+            const int meta = vmisc[kMiscMeta + slot];
+            if (meta == kItemEnd) return false;
+            const int kind = item_kind(meta);
+            int u, part, slot0, n;
+            if (kind == kKindExtra) {
+                const int i = meta & 0xfffffff;
+                u = i / nsl;
+                part = i % nsl;
+                slot0 = Tk + u * kFTile;
+                n = T - u * kFTile < kFTile ? T - u * kFTile : kFTile;
+            } else {
+                const int ug0 = staged ? nsh : 0;
+                if (kind == kKindGU) {
+                    const int it = meta & 0xfffffff;
+                    u = ug0 + it / nsl;
+                    part = it % nsl;
+                } else {
+                    const int d = meta & 0xfffff;
+                    u = d / ndn;
+                    part = d % ndn;
+                }
+                const int4 un = units[u];
+                slot0 = un.y;
+                n = un.z;
+            }
+            const uint8_t *w = ring + (size_t)slot * p.item_bytes;
+            float *rd = red + (size_t)slot * (kRedSlot / 4);  // [warp of group][lane][8]
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+            if (kind != kKindDown) {
+                // ---------------------------------- gate/up slab, K eighth q
+                // pairs of blocks: every range starts at an even block
+                const int b0 = 2 * (q * (nbh / 2) / 8), b1 = 2 * ((q + 1) * (nbh / 2) / 8);
+                // the lane's two token columns (columns past n repeat token 0)
+                const int ta = slot_tok(slot0 + (2 * cq < n ? 2 * cq : 0));
+                const int tb = slot_tok(slot0 + (2 * cq + 1 < n ? 2 * cq + 1 : 0));
+                if constexpr (kStaged) {
+                    const int r = lane & 7;
+                    const __half *rowp = xs + (size_t)slot_tok(slot0 + (r < n ? r : 0)) * (H + 8);
+                    slab2_blocks<kBits, kSrcSmem, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
+                                                          scorr + ta * nbh, scorr + tb * nbh, lane);
+                } else {
+                    const __half *rowp = p.x16 + (size_t)slot_tok(slot0 + (g < n ? g : 0)) * H;
+                    slab2_blocks<kBits, kSrcLdg, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
+                                                         p.corr + (size_t)ta * nbh,
+                                                         p.corr + (size_t)tb * nbh, lane);
+                }
+                float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
+                rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+                rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
+                __syncwarp();
+                if (!last_warp(slot)) {
+                    if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
+                    continue;
+                }
+                // the last warp: the K eighths in a fixed order, then SwiGLU
+                float gs[4] = {0.f, 0.f, 0.f, 0.f}, us[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < kGWarps; j++) {
+                    const float4 *rj = reinterpret_cast<const float4 *>(rd + ((size_t)j * 32 + lane) * 8);
+                    const float4 vg = rj[0], vu = rj[1];
+                    gs[0] += vg.x; gs[1] += vg.y; gs[2] += vg.z; gs[3] += vg.w;
+                    us[0] += vu.x; us[1] += vu.y; us[2] += vu.z; us[3] += vu.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);  // weights and partials consumed
+                // undo the operand factor: 2^8 (magic-offset form) or 2 (exact integers)
+                const float back = kMagic ? 1.0f / 256.0f : 0.5f;
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
-                    float gs = ((r0[i] + r1[i]) + r2[i]) + r3[i];
-                    float us = ((r0[4 + i] + r1[4 + i]) + r2[4 + i]) + r3[4 + i];
-                    gs *= 0.5f;  // the integers are 2(q - c): one factor 2 out
-                    us *= 0.5f;
-                    const float av = gs / (1.0f + expf(-gs)) * us;
                     const int tok = 2 * cq + (i & 1);
+                    const float gv = gs[i] * back, uv = us[i] * back;
+                    // silu of the true gate value; the product stays in the
+                    // token's prescaled units (times 2^-2ex)
+                    const int ex = tok < n ? slot_exp(slot0 + tok) : 0;
+                    const float gt = ex ? gv * pow2f(ex) : gv;
+                    const float av = gv / (1.0f + expf(-gt)) * uv;
                     const int row = part * kSlabRows + g + 8 * (i >> 1);
                     if (tok < n) p.a[(size_t)(slot0 + tok) * p.Ip + row] = __float2half_rn(av);
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    __threadfence();  // the warp's stores, then the count
-                    atomicAdd(p.done_gu + u, 1);
+                    // post the slab's unit for the publish warp (CTA scope)
+                    __threadfence_block();
+                    const int idx = atomicAdd(misc + kMiscPubN, 1);
+                    long long t0 = clock64();
+                    while (idx - vmisc[kMiscPubSeen] >= kPubQ) {
+                        if (*abort_flag || clock64() - t0 > p.budget) {
+                            atomicCAS(p.err, 0, kErrTimeout);
+                            *abort_flag = 1;
+                            break;
+                        }
+                    }
+                    vmisc[kMiscPubQ + idx % kPubQ] = u + 1;
                 }
-            }
-            group_sync(gi);  // the reduction scratch is free again
-        } else {
-            // --------------------------------------------------- down item
-            const int ar = lane & 7;
-            const __half *rowp = abuf + (size_t)(ar < n ? ar : 0) * (p.Ip + 8);
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            const uint8_t *w0 = w + (size_t)(2 * q) * p.nseg_i * UB;  // slabs 2q, 2q + 1
-            fused_slab2<kBits, kSrcSmem>(acc[0], acc[1], w0, w0 + (size_t)p.nseg_i * UB, p.nseg_i,
-                                         rowp, 0, lane);
-#pragma unroll
-            for (int s = 0; s < 2; s++)
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int tok = 2 * cq + (i & 1);
-                    const int row = (part * kDownSlabs + 2 * q + s) * kSlabRows + g + 8 * (i >> 1);
-                    if (tok < n) p.Y[(size_t)(slot0 + tok) * H + row] = 0.5f * acc[s][i];
+            } else {
+                // ------------------ down block: slabs 2 (q >> 1) + {0, 1}, K half q & 1
+                const int kd = (meta >> 20) & 0xff, b = kd % p.na;
+                if (!warp_fwait(&abar[b], (kd / p.na) & 1, p, abort_flag, lane)) return false;
+                const __half *abuf = abuf0 + (size_t)b * kFTile * (p.Ip + 8);
+                const int ar = lane & 7, pr = q >> 1, h = q & 1;
+                const __half *rowp = abuf + (size_t)(ar < n ? ar : 0) * (p.Ip + 8);
+                const uint8_t *s0 = w + (size_t)(2 * pr) * p.nseg_i * UB;
+                slab2_blocks<kBits, kSrcSmem, false>(a0, a1, s0, s0 + (size_t)p.nseg_i * UB,
+                                                     2 * (h * (nbi / 2) / 2), 2 * ((h + 1) * (nbi / 2) / 2), rowp, nullptr,
+                                                     nullptr, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aempty[b]);  // activation rows consumed
+                float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
+                rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+                rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
+                __syncwarp();
+                if (!last_warp(slot)) {
+                    if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
+                    continue;
                 }
-            __threadfence();
-            group_sync(gi);
-            if (gtid == 0) {
-                mbar_arrive(&empty[slot]);
-                int nc = 0;
-                for (int i = 0; i < n; i++) {
-                    const int sl = slot0 + i;
-                    const int t = sl < Tk ? slist[sl] : sl - Tk;
-                    if (atomicAdd(p.done_tok + t * ndn + part, 1) == per_blk - 1)
-                        comb[1 + nc++] = t;
+                // the last warp: both K halves of every slab, in a fixed order
+#pragma unroll
+                for (int pp = 0; pp < kDownSlabs / 2; pp++) {
+                    const float4 *r0 = reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp) * 32 + lane) * 8);
+                    const float4 *r1 =
+                        reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp + 1) * 32 + lane) * 8);
+#pragma unroll
+                    for (int sl = 0; sl < 2; sl++) {
+                        const float4 v0 = r0[sl], v1 = r1[sl];
+                        const float yv[4] = {v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w};
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            const int tok = 2 * cq + (i & 1);
+                            const int row = (part * kDownSlabs + 2 * pp + sl) * kSlabRows + g + 8 * (i >> 1);
+                            if (tok < n) p.Y[(size_t)(slot0 + tok) * H + row] = 0.5f * yv[i];
+                        }
+                    }
                 }
-                comb[0] = nc;
-                __threadfence();
-            }
-            group_sync(gi);
-            // this item finished the last expert rows of these (token, block)
-            // pairs: y = Y_shared + sum over the picks in ascending expert id
-            // of w Y, one column per thread, every row requested up front
-            for (int ci = 0; ci < comb[0]; ci++) {
-                const int t = comb[1 + ci];
-                const int col = part * kSlabRows * kDownSlabs + gtid;
-                float v[kFMaxK];
-#pragma unroll
-                for (int r = 0; r < kFMaxK; r++)
-                    v[r] = r < k ? __ldcg(p.Y + (size_t)sslot[sord[t * k + r]] * H + col) : 0.0f;
-                float acc = __ldcg(p.Y + (size_t)(Tk + t) * H + col);
-#pragma unroll
-                for (int r = 0; r < kFMaxK; r++)
-                    if (r < k) acc = fmaf(sw[sord[t * k + r]], v[r], acc);
-                __nv_bfloat16 *o = p.out + (size_t)t * H + col;
-                const __nv_bfloat16 yb = __float2bfloat16_rn(acc);
-                *o = p.residual ? __float2bfloat16_rn(__fadd_rn(__bfloat162float(*o),
-                                                                __bfloat162float(yb)))
-                                : yb;
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty[slot]);  // weights and partials consumed
+                    // all 128 rows are stored: post the block for the combine warp
+                    __threadfence_block();
+                    const int idx = atomicAdd(misc + kMiscCombN, 1);
+                    long long t0 = clock64();
+                    while (idx - vmisc[kMiscCombSeen] >= kPubQ) {
+                        if (*abort_flag || clock64() - t0 > p.budget) {
+                            atomicCAS(p.err, 0, kErrTimeout);
+                            *abort_flag = 1;
+                            break;
+                        }
+                    }
+                    vmisc[kMiscCombQ + idx % kPubQ] = u * ndn + part + 1;
+                }
             }
         }
+        return true;
+    };
+
+    // ---- the shared expert's slabs (no routing needed) while the grid barrier runs
+    if (alive) alive = run_items(nwc + nx);
+    // one verdict for all compute warps before the next compute-wide barriers
+    // (a warp that gave up above must not skip a barrier the others wait at)
+    if (!alive) misc[kMiscDead] = 1;
+    compute_sync();
+    alive = misc[kMiscDead] == 0;
+
+    // ---- top-k (picks in descending logit order; a tie to the lower id)
+    if (tid == 0) *cflag = alive && fwait(rdy, 0, p, abort_flag) ? 1 : 0;
+    compute_sync();
+    alive = *cflag != 0;
+    if (T <= kTopkLocalT) {
+        if (alive && warp < T) {
+            int pe;
+            float pw;
+            warp_topk(p.logits + (size_t)warp * E, E, k, lane, pe, pw);
+            if (lane < k) {
+                sidx[warp * k + lane] = pe;
+                sw[warp * k + lane] = pw;
+            }
+        }
+    } else {
+        if (alive && warp == 0 && cta < T) {
+            int pe;
+            float pw;
+            warp_topk(p.logits + (size_t)cta * E, E, k, lane, pe, pw);
+            if (lane < k) {
+                p.idx[(size_t)cta * k + lane] = pe;
+                p.wts[(size_t)cta * k + lane] = pw;
+            }
+        }
+        __syncwarp();
+        compute_sync();
+        if (tid == 0) {
+            mbar_arrive(pickbar);
+            *cflag = alive && fwait(rdy2, 0, p, abort_flag) ? 1 : 0;
+        }
+        compute_sync();
+        alive = *cflag != 0;
+        if (alive)
+            for (int i = tid; i < Tk; i += kFCompute) {
+                sidx[i] = __ldcg(p.idx + i);
+                sw[i] = __ldcg(p.wts + i);
+            }
+    }
+    compute_sync();
+
+    // ---- dispatch, identical in every CTA
+    if (alive) {
+        for (int i = tid; i < Tk; i += kFCompute) atomicOr(&mask[sidx[i]], 1ull << (i / k));
+        compute_sync();
+        // one scan of (count << 16 | units): both sums stay below 2^16 (T k <= 1024)
+        const int ept = (E + kFCompute - 1) / kFCompute, eb = tid * ept;
+        int local = 0;
+        for (int e = eb; e < eb + ept && e < E; e++) {
+            const int c = __popcll(mask[e]);
+            local += (c << 16) | ((c + kFTile - 1) / kFTile);
+        }
+        int packed_total;
+        int packed = compute_exclusive_scan(local, misc + kMiscScan, &packed_total);
+        const int utot = packed_total & 0xffff;
+        for (int e = eb; e < eb + ept && e < E; e++) {
+            const int c = __popcll(mask[e]), nu = (c + kFTile - 1) / kFTile;
+            const int off = packed >> 16, us = packed & 0xffff;
+            soff[e] = off;
+            for (int i = 0; i < nu; i++) {
+                const int n = c - i * kFTile;
+                units[nsh + us + i] = make_int4(e, off + i * kFTile, n < kFTile ? n : kFTile, 0);
+            }
+            packed += (c << 16) | nu;
+        }
+        if (tid < nsh) {
+            const int n = T - tid * kFTile;
+            units[tid] = make_int4(E, Tk + tid * kFTile, n < kFTile ? n : kFTile, 0);
+        }
+        if (tid == 0) {
+            misc[kMiscNUnits] = nsh + utot;
+            misc[kMiscUtot] = utot;
+        }
+        compute_sync();
+        for (int i = tid; i < Tk; i += kFCompute) {
+            const int t = i / k, ej = sidx[i];
+            const int pos = soff[ej] + __popcll(mask[ej] & ((1ull << t) - 1ull));
+            slist[pos] = t;
+            sslot[i] = pos;
+            int rank = 0;
+            for (int jj = 0; jj < k; jj++) rank += sidx[t * k + jj] < ej;
+            sord[t * k + rank] = i;  // combine order: ascending expert id
+        }
+    }
+    compute_sync();
+    if (tid == 0 && alive) mbar_arrive(dsp);
+    // the next kernel of the stream may start its prologue once every CTA is here
+    grid_launch_dependents();
+
+    // ---- routed slabs and down blocks, then the end marker
+    if (alive) run_items(1 << 30);
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(misc + kMiscWarpsDone, 1);  // the publish warp may stop once all are in
     }
 }
 
@@ -553,8 +1236,8 @@ static int g_fused_max_smem = 0;
 static int g_fused_sms = 0;
 
 int fused_decode_supported(const Geometry &g, int T) {
-    return T >= 1 && T <= kFMaxT && g.E <= 512 && g.E <= 2 * kFThreads && g.k <= kFMaxK &&
-           g.H % 128 == 0 && g.Ip % 128 == 0 && g.H <= 8192;
+    return T >= 1 && T <= kFMaxT && g.E <= 512 && g.k <= kFMaxK && g.H % 128 == 0 &&
+           g.Ip % 128 == 0 && g.H <= 8192;
 }
 
 size_t fused_item_bytes(const Geometry &g) {
@@ -562,20 +1245,19 @@ size_t fused_item_bytes(const Geometry &g) {
     return (size_t)(a > b ? a : b) * g.ub;
 }
 
-cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const int32_t *idx,
-                                const float *wts, const void *x16, int T, int units_max, void *a,
-                                float *Y,
-                                void *out, bool residual, int *done_gu, int *done_tok, int *queue,
-                                int *err, long long budget, cudaStream_t s) {
+int fused_grid() { return g_fused_sms; }
+
+cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const FusedArgs &fa,
+                                int T, cudaStream_t s) {
     if (!fused_decode_supported(g, T) || g_fused_max_smem == 0) return cudaErrorInvalidValue;
     FusedParams p{};
+    p.x = reinterpret_cast<const __nv_bfloat16 *>(fa.x);
+    p.Wp = reinterpret_cast<const float4 *>(fa.router_wp);
+    p.bias = fa.router_b;
     p.routed = w.routed;
     p.shared = w.shared;
     p.expert_bytes = g.expert_bytes;
     p.mat_bytes = g.mat_bytes;
-    p.idx = idx;
-    p.wts = wts;
-    p.x16 = reinterpret_cast<const __half *>(x16);
     p.T = T;
     p.E = g.E;
     p.k = g.k;
@@ -584,30 +1266,66 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     p.nseg_h = g.nseg_h;
     p.nseg_i = g.nseg_i;
     p.item_bytes = (int)fused_item_bytes(g);
-    p.units_max = units_max;
-    p.a = reinterpret_cast<__half *>(a);
-    p.Y = Y;
-    p.out = reinterpret_cast<__nv_bfloat16 *>(out);
-    p.residual = residual ? 1 : 0;
-    p.done_gu = done_gu;
-    p.done_tok = done_tok;
-    p.queue = queue;
-    p.err = err;
-    p.budget = budget;
-    // ring depth and token staging from the shared memory left over
-    const int fixed_nost =
-        fused_smem(T, g.E, g.k, g.H, g.Ip, 0, p.item_bytes, 0, units_max).total;
+    p.units_max = max_units(T, g.k, g.E, kFTile);
+    p.cnt_tok = fa.cnt_tok;
+    p.w2 = fa.w2;
+    p.logits = fa.logits;
+    p.idx = fa.idx;
+    p.wts = fa.wts;
+    p.x16 = reinterpret_cast<__half *>(fa.x16);
+    p.corr = fa.corr;
+    p.xex = fa.xex;
+    p.a = reinterpret_cast<__half *>(fa.a);
+    p.Y = fa.Y;
+    p.out = reinterpret_cast<__nv_bfloat16 *>(fa.out);
+    p.residual = fa.residual ? 1 : 0;
+    p.bar = fa.bar;
+    p.cnt = fa.cnt;
+    p.cnt_stride = fa.cnt_stride;
+    p.err = fa.err;
+    p.budget = fa.budget;
+    const int G = g_fused_sms;
+    // the router slice of the CTA with the most experts must fit the ring
+    const int ne_max = (g.E + G - 1) / G;
+    const int wb = ne_max * g.H * 4;
+    // shared memory: staging of the token rows, then activation buffers and
+    // as deep a ring as fits
     const int xs_bytes = align16(T * (g.H + 8) * 2);
-    p.staged = (T <= kFStagedMaxT && g_fused_max_smem - fixed_nost - xs_bytes >= 4 * p.item_bytes)
+    auto total = [&](int ring, int staged, int na) {
+        return fused_smem(T, g.E, g.k, g.H, g.Ip, ring, p.item_bytes, staged, p.units_max, na)
+            .total;
+    };
+    // a ring slot costs its item bytes plus the partial sums of the warps; the
+    // partial-sum area also holds the router's copy of staged token rows
+    const int slot_bytes = p.item_bytes + kRedSlot;
+    const int xi_slots = (align16(T * g.H * 2) + kRedSlot - 1) / kRedSlot;
+    p.na = 2;
+    p.staged = (T <= kFStagedMaxT && g_fused_max_smem - total(0, 1, p.na) >=
+                                         (xi_slots > 4 ? xi_slots : 4) * slot_bytes)
                    ? 1 : 0;
-    const int room = g_fused_max_smem - fixed_nost - (p.staged ? xs_bytes : 0);
-    p.ring = room / p.item_bytes;
+    (void)xs_bytes;
+    const int room = g_fused_max_smem - total(0, p.staged, p.na);
+    p.ring = room / slot_bytes;
     if (p.ring > kFMaxRing) p.ring = kFMaxRing;
-    if (p.ring < 2) return cudaErrorInvalidValue;
-    const int smem =
-        fused_smem(T, g.E, g.k, g.H, g.Ip, p.ring, p.item_bytes, p.staged, units_max).total;
-    auto kern = g.bits == 2 ? fused_decode_kernel<2> : fused_decode_kernel<3>;
-    return launch_pdl(kern, dim3(g_fused_sms), dim3(kFThreads), (size_t)smem, s, p);
+    if (p.staged && p.ring < xi_slots) return cudaErrorInvalidValue;
+    const int nwc = (wb + p.item_bytes - 1) / p.item_bytes;
+    if (p.ring < 2 || nwc >= p.ring) return cudaErrorInvalidValue;
+    const int smem = total(p.ring, p.staged, p.na);
+    auto kern = g.bits == 2 ? (p.staged ? fused_decode_kernel<2, true> : fused_decode_kernel<2, false>)
+                            : (p.staged ? fused_decode_kernel<3, true> : fused_decode_kernel<3, false>);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kFThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;  // the CTAs wait on one another
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 cudaError_t fused_init_attributes(int max_smem) {
@@ -615,10 +1333,12 @@ cudaError_t fused_init_attributes(int max_smem) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&g_fused_sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t e;
-    if ((e = allow_max_dyn_smem(fused_decode_kernel<2>, max_smem)) != cudaSuccess) return e;
-    if ((e = allow_max_dyn_smem(fused_decode_kernel<3>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<2, true>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<2, false>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<3, true>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<3, false>, max_smem)) != cudaSuccess) return e;
     cudaFuncAttributes fa;
-    if ((e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(fused_decode_kernel<2>))) !=
+    if ((e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(fused_decode_kernel<2, true>))) !=
         cudaSuccess)
         return e;
     g_fused_max_smem = max_smem - (int)fa.sharedSizeBytes;
@@ -626,4 +1346,3 @@ cudaError_t fused_init_attributes(int max_smem) {
 }
 
 }  // namespace strata
-

@@ -29,14 +29,8 @@ void launch_debug_dequant(const uint8_t *mat, int bits, int Kp, int row0, int nr
 
 // ---- route.cu
 // Router weight in the lane-interleaved layout: Wp[e][H/128][32 lanes][4].
-// For the fused decode kernel that follows (all optional): x16, the fp16 copy
-// of x [T][H]; zero, nzero ints zeroed; tok_done (one counter per group of up
-// to 8 tokens, zero between launches): the top-k of every token written to
-// idx / w [T][k] by the last CTA of its token group.
 void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                   float *logits, cudaStream_t s, void *x16 = nullptr, int *zero = nullptr,
-                   int nzero = 0, int k = 0, int32_t *idx = nullptr, float *w = nullptr,
-                   int *tok_done = nullptr);
+                   float *logits, cudaStream_t s);
 void launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
                  cudaStream_t s);
 
@@ -106,16 +100,33 @@ void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s);
 cudaError_t umma_init_attributes(int max_smem);
 
 // ---- decode.cu (fused decode layer, T <= 64)
-// After launch_router(..., x16, counters, units_max + T (H / 128), k, idx, w,
-// tok_done): dispatch, gate/up, down and combine in one kernel (programmatic
-// dependent launch).
-// done_gu [units_max], done_tok [T][H / 128] and queue [2] are router-zeroed counters.
+// The whole layer in one cooperative launch (router, top-k, dispatch,
+// gate/up, down, combine); see decode.cu.
+struct FusedArgs {
+    const void *x;              // bf16 [T][H] layer input
+    const float *router_wp;     // lane-interleaved router weight
+    const float *router_b;      // [E] or null
+    float w2;                   // token prescale bound (0: none)
+    float *logits;              // [T][E]
+    int32_t *idx;               // [T][k]
+    float *wts;                 // [T][k]
+    void *x16;                  // fp16 [T][H] expert token operand
+    float *corr;                // [T][H / 32] its block corrections (2-bit)
+    int *xex;                   // [T]
+    void *a;                    // fp16 [slots][Ip]
+    float *Y;                   // fp32 [slots][H]
+    void *out;                  // bf16 [T][H]
+    bool residual;              // out <- bf16(out + y) instead of out <- y
+    unsigned long long *bar;    // grid barrier counter (zero at create, never reset)
+    int *cnt;                   // 2 counter sets (zero at create)
+    int cnt_stride;             // ints per set: cnt_tok + 64 * (H / 128)
+    int cnt_tok;                // max_units(64, k, E, 8): per-unit counters come first
+    int *err;
+    long long budget;
+};
 int fused_decode_supported(const Geometry &g, int T);
-cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const int32_t *idx,
-                                const float *wts, const void *x16, int T, int units_max, void *a,
-                                float *Y,
-                                void *out, bool residual, int *done_gu, int *done_tok, int *queue,
-                                int *err, long long budget, cudaStream_t s);
+cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const FusedArgs &a,
+                                int T, cudaStream_t s);
 cudaError_t fused_init_attributes(int max_smem);
 
 // ---- combine.cu

@@ -21,124 +21,23 @@
 
 namespace strata {
 
-// ============================================================== warp top-k
-// Order-preserving 32-bit key of a logit: larger float <=> larger key; -0 is
-// read as +0 (equal floats, equal keys) and a NaN as -inf (it ranks last).
-// Key 0 is below every logit and marks a taken or missing entry.
-__device__ __forceinline__ uint32_t logit_key(float f) {
-    if (f != f) f = -INFINITY;
-    if (f == 0.0f) f = 0.0f;
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_logit(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Best of a lane's 16 entries: the largest key, and on equal keys the lowest
-// q.  A pairwise tree over adjacent entries: the left operand of every
-// comparison holds the lower q's, so ">=" keeps ties on the lower q.
-__device__ __forceinline__ void lane_best(const uint32_t (&key)[16], uint32_t &bk, int &bq) {
-    uint32_t k8[8], k4[4], k2[2];
-    int q8[8], q4[4], q2[2];
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const bool l = key[2 * i] >= key[2 * i + 1];
-        k8[i] = l ? key[2 * i] : key[2 * i + 1];
-        q8[i] = l ? 2 * i : 2 * i + 1;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const bool l = k8[2 * i] >= k8[2 * i + 1];
-        k4[i] = l ? k8[2 * i] : k8[2 * i + 1];
-        q4[i] = l ? q8[2 * i] : q8[2 * i + 1];
-    }
-#pragma unroll
-    for (int i = 0; i < 2; i++) {
-        const bool l = k4[2 * i] >= k4[2 * i + 1];
-        k2[i] = l ? k4[2 * i] : k4[2 * i + 1];
-        q2[i] = l ? q4[2 * i] : q4[2 * i + 1];
-    }
-    const bool l = k2[0] >= k2[1];
-    bk = l ? k2[0] : k2[1];
-    bq = l ? q2[0] : q2[1];
-}
-
-// Top-k of one token by one warp (E <= 512: lane l holds logits l, l+32, ...).
-// Each round takes the largest key over the warp (redux.sync max) and, among
-// the lanes holding it, the lowest expert id (redux.sync min), i.e. the larger
-// logit and on equal logits the lower id; the winning lane drops that entry
-// and finds its next best.  Lane j < k ends with pick j and its weight
-// exp(l_j - m) / sum.
-__device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
-                                        int &pick_e, float &pick_w) {
-    uint32_t key[16];
-    const int nq = (E + 31) >> 5;
-#pragma unroll
-    for (int q = 0; q < 16; q++) {
-        const int e = q * 32 + lane;
-        key[q] = (q < nq && e < E) ? logit_key(__ldcg(row + e)) : 0u;
-    }
-    uint32_t bk;
-    int bq;
-    lane_best(key, bk, bq);
-    uint32_t my_k = 0u;
-    int my_e = -1;
-    for (int j = 0; j < k; j++) {
-        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t cand = (bk == wk && bk != 0u) ? (uint32_t)(bq * 32 + lane) : 0xffffffffu;
-        const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
-        if (lane == j) {
-            my_k = wk;
-            my_e = (int)we;
-        }
-        if ((int)(we & 31u) == lane) {
-            const int wq = (int)(we >> 5);
-#pragma unroll
-            for (int q = 0; q < 16; q++) key[q] = q == wq ? 0u : key[q];
-            lane_best(key, bk, bq);
-        }
-    }
-    const float my_v = key_logit(my_k);
-    const float m = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = lane < k ? expf(my_v - m) : 0.0f;
-    float sum = ex;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    pick_e = my_e;
-    pick_w = ex / sum;
-}
-
 // ============================================================== router
 // CTA: NW warps; warp owns EE experts, lanes are the 32 residue classes of the
 // fixed order; TT tokens per CTA staged in shared memory as bf16 in the same
 // lane-interleaved layout as the weights: xs[tt][s4][lane] holds the 4 values
 // x[128*s4 + 32*j + lane], j = 0..3 (8 bytes, so the staging stores and the
 // LDS.64 reads are conflict-free; widening bf16 to fp32 is exact).
-// Optional side outputs for the fused decode kernel that follows: x16 (fp16
-// copy of x, written by the CTAs of expert block 0), nzero ints zeroed, and
-// the top-k picks: with tok_done set, the last CTA to finish a token group
-// (a counter per group, reset by that CTA) runs the top-k of its tokens and
-// writes idx / wout, so the next kernel reads T k picks, not T E logits.
 template <int TT, int EE, int CH, int NW>
 __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__restrict__ x, int T,
                                                      int H, const float4 *__restrict__ Wp,
                                                      const float *__restrict__ bias, int E,
-                                                     float *__restrict__ logits,
-                                                     __half *__restrict__ x16,
-                                                     int *__restrict__ zero, int nzero, int k,
-                                                     int32_t *__restrict__ idx,
-                                                     float *__restrict__ wout,
-                                                     int *__restrict__ tok_done) {
+                                                     float *__restrict__ logits) {
     extern __shared__ uint2 xs[];
     // a dependent kernel may be scheduled now; it waits for this grid's
     // completion before reading anything written here
     grid_launch_dependents();
     const int ns4 = H / 128;
     const int t0 = blockIdx.y * TT;
-    if (zero && blockIdx.x == 0 && blockIdx.y == 0)
-        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
-    const bool write16 = x16 != nullptr && blockIdx.x == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e0 = (blockIdx.x * NW + warp) * EE;
     // the first CH steps of this warp's weights are requested before the
@@ -180,16 +79,10 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
             const int sl = base + b * blockDim.x + threadIdx.x;
             if (sl >= nslot) break;
             xs[sl] = make_uint2(v[b][0] | (v[b][1] << 16), v[b][2] | (v[b][3] << 16));
-            const int tt = sl / (ns4 * 32), r = sl % (ns4 * 32);
-            if (write16 && t0 + tt < T) {
-                __half *o = x16 + (size_t)(t0 + tt) * H + (r >> 5) * 128 + (r & 31);
-#pragma unroll
-                for (int j = 0; j < 4; j++) o[32 * j] = __float2half_rn(__uint_as_float(v[b][j] << 16));
-            }
         }
     }
     __syncthreads();
-    if (e0 < E) {
+    if (e0 >= E) return;
     float acc[TT][EE];
 #pragma unroll
     for (int a = 0; a < TT; a++)
@@ -241,57 +134,28 @@ __global__ __launch_bounds__(32 * NW) void router_kernel(const __nv_bfloat16 *__
             }
         }
     }
-    }
-    if (tok_done == nullptr) return;
-    __shared__ int s_last;
-    // One gpu-scope acquire-release add per CTA: its release half publishes
-    // the logits this CTA stored (the barrier before it orders every warp's
-    // stores first), and in the last CTA of the token group its acquire half,
-    // extended to the other warps by the barrier after it, makes every other
-    // CTA's logits visible to the loads of the top-k.
-    __syncthreads();
-    if (threadIdx.x == 0)
-        s_last = atom_add_acq_rel_gpu(tok_done + blockIdx.y, 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    for (int a = warp; a < TT; a += NW) {
-        const int t = t0 + a;
-        if (t >= T) break;
-        int pe;
-        float pw;
-        warp_topk(logits + (size_t)t * E, E, k, lane, pe, pw);
-        if (lane < k) {
-            idx[(size_t)t * k + lane] = pe;
-            wout[(size_t)t * k + lane] = pw;
-        }
-    }
-    if (threadIdx.x == 0) tok_done[blockIdx.y] = 0;  // ready for the next launch
 }
 
 template <int TT, int EE, int CH, int NW>
 static void run_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                       float *logits, void *x16, int *zero, int nzero, int k, int32_t *idx,
-                       float *w, int *tok_done, cudaStream_t s) {
+                       float *logits, cudaStream_t s) {
     size_t smem = (size_t)TT * H * sizeof(__nv_bfloat16);
     auto kern = router_kernel<TT, EE, CH, NW>;
     dim3 grid((E + NW * EE - 1) / (NW * EE), (T + TT - 1) / TT);
     kern<<<grid, 32 * NW, smem, s>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
-                                 reinterpret_cast<const float4 *>(Wp), bias, E, logits,
-                                 reinterpret_cast<__half *>(x16), zero, nzero, k, idx, w,
-                                 tok_done);
+                                 reinterpret_cast<const float4 *>(Wp), bias, E, logits);
 }
 
 void launch_router(const void *x, int T, int H, const float *Wp, const float *bias, int E,
-                   float *logits, cudaStream_t s, void *x16, int *zero, int nzero, int k,
-                   int32_t *idx, float *w, int *tok_done) {
+                   float *logits, cudaStream_t s) {
     if (T <= 1)
-        run_router<1, 1, 20, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<1, 1, 20, 4>(x, T, H, Wp, bias, E, logits, s);
     else if (T <= 4)
-        run_router<4, 1, 20, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<4, 1, 20, 4>(x, T, H, Wp, bias, E, logits, s);
     else if (T <= 64)
-        run_router<8, 2, 8, 8>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<8, 2, 8, 8>(x, T, H, Wp, bias, E, logits, s);
     else
-        run_router<8, 8, 2, 4>(x, T, H, Wp, bias, E, logits, x16, zero, nzero, k, idx, w, tok_done, s);
+        run_router<8, 8, 2, 4>(x, T, H, Wp, bias, E, logits, s);
 }
 
 // ============================================================== top-k

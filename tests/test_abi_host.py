@@ -93,7 +93,17 @@ def test_config_struct_layout_matches_header():
 
 
 def test_weights_struct_points_into_arrays():
+    """Every pointer of the weights struct is the data of the kept array of the
+    same field, and each kept array holds the layer's values in the C types the
+    header declares (the tiny layer has no router bias, so router_b is NULL)."""
     layer = gen.layer_weights(gen.TINY, seed=0)
     w, keep = qe.make_weights(layer)
-    assert w.codes == keep[0].ctypes.data and w.router_b is None
-    assert np.shares_memory(keep[0], layer.codes) or keep[0].base is not None or True
+    fields = ["codes", "scales", "router_w", "router_b", "shared_codes", "shared_scales"]
+    dtypes = [np.uint8, np.uint16, np.float32, np.float32, np.uint8, np.uint16]
+    assert layer.router_b is None and w.router_b is None and keep[3] is None
+    for name, a, dt in zip(fields, keep, dtypes):
+        if a is None:
+            continue
+        assert getattr(w, name) == a.ctypes.data, name
+        assert a.dtype == dt and a.flags.c_contiguous, name
+        assert np.array_equal(a.reshape(-1), np.asarray(getattr(layer, name)).reshape(-1)), name

@@ -215,9 +215,11 @@ def test_forward_host_pinned():
     assert np.array_equal(host(xa, ya, 4), device_ref(xa, 4))
     qe.strata_moe_set_option(L.handle, qe.STRATA_OPT_PATH, 1)  # the decode kernel chain
     y_chain = host(xa, ya, 4)
-    qe.strata_moe_set_option(L.handle, qe.STRATA_OPT_PATH, 0)
     assert np.array_equal(y_chain, device_ref(xa, 4))
-    assert np.array_equal(host(xa, ya, 4), y_chain)
+    qe.strata_moe_set_option(L.handle, qe.STRATA_OPT_PATH, 0)  # back to the fused kernel
+    y_fused = host(xa, ya, 4)
+    assert np.array_equal(y_fused, device_ref(xa, 4))
+    close_outputs(y_fused, y_chain, "host forward, fused vs chain")
 
 
 def test_zero_and_oversized_batches():
@@ -324,13 +326,26 @@ def _tie_layers(shape, seed):
     return out
 
 
+def close_outputs(a_bits, b_bits, label):
+    """Two bf16 layer outputs of the same input that differ only by rounding:
+    every element within 2^-8 of the largest magnitude (about one bf16 unit in
+    the last place of the largest element) and the mean difference within
+    1e-3 of the mean magnitude."""
+    a, b = npref.bf16_bits_to_f64(a_bits), npref.bf16_bits_to_f64(b_bits)
+    err = np.abs(a - b)
+    assert err.max() <= 2.0 ** -8 * np.abs(b).max(), f"{label}: max diff {err.max():.3e}"
+    assert err.sum() <= 1e-3 * np.abs(b).sum(), f"{label}: mean diff {err.sum() / np.abs(b).sum():.3e}"
+
+
 @pytest.mark.parametrize("T", [1, 4, 13, 64])
-def test_fused_decode_equals_gemv_chain(T):
-    """The fused decode kernel (router top-k in the router's last CTA, dispatch,
-    gate/up, down and combine in one launch) does the same arithmetic in the
-    same order as the chain of decode kernels, so the two outputs are equal bit
-    for bit, also where the routing meets exact ties and one-ulp near-ties;
-    and both match the oracle."""
+def test_fused_decode_agrees_with_gemv_chain(T):
+    """The fused decode kernel (router, top-k, dispatch, gate/up, down and
+    combine in one launch) against the chain of decode kernels on exact ties,
+    one-ulp near-ties and an all-zero router: the same routing (both equal to
+    the oracle's, bit for bit), both outputs within the layer tolerance of the
+    oracle, and the two outputs equal up to rounding (the fused kernel's
+    gate/up products use the magic-offset form and sum its K splits in its own
+    fixed order, so the fp32 values may round to neighbouring bf16 values)."""
     shape = gen.LayerShape(hidden=512, n_experts=512, top_k=10, inter=128, bits=2,
                            router_bias=True)
     for label, w in _tie_layers(shape, seed=41):
@@ -340,23 +355,31 @@ def test_fused_decode_equals_gemv_chain(T):
         fused.set_option(qe.STRATA_OPT_PATH, 3)
         chain = qe.Layer(w, max_tokens=T)
         chain.set_option(qe.STRATA_OPT_PATH, 1)
-        assert qe.strata_moe_launch_count(fused.handle, T) == 2
+        assert qe.strata_moe_launch_count(fused.handle, T) == 1
         yf = from_dev_bf16(fused.forward(xt))
         yc = from_dev_bf16(chain.forward(xt))
         fused.sync_status()
         chain.sync_status()
-        assert np.array_equal(yf, yc), f"T={T} {label}: fused and chained outputs differ"
+        check_route(fused, w, x, T, f"fused T={T} {label}")
         _, ref, _, _ = oracle.moe_forward(w, x, threads=THREADS)
         check_output(yf, ref, f"fused T={T} {label}")
+        check_output(yc, ref, f"chain T={T} {label}")
+        close_outputs(yf, yc, f"fused vs chain T={T} {label}")
 
 
 def test_fused_decode_3bit_batch():
-    """3-bit weights at the batched-decode size, fused against the chain."""
+    """3-bit weights at the batched-decode size: fused against the chain and
+    the oracle."""
     shape, T = gen.FLASH3, 64
-    x = to_dev_bf16(gen.hidden(T, shape.hidden, seed=43))
+    xh = gen.hidden(T, shape.hidden, seed=43)
+    x = to_dev_bf16(xh)
     fused = gpu_layer(shape, T, path=3)
     chain = gpu_layer(shape, T, path=1)
     yf = from_dev_bf16(fused.forward(x))
     yc = from_dev_bf16(chain.forward(x))
     fused.sync_status()
-    assert np.array_equal(yf, yc)
+    chain.sync_status()
+    close_outputs(yf, yc, "fused vs chain 3-bit T=64")
+    sel = np.arange(0, T, 3, dtype=np.int32)
+    _, ref, _, _ = oracle.moe_forward(layer_of(shape), xh, sel=sel, threads=THREADS)
+    check_output(yf[sel], ref, "fused 3-bit T=64")
