@@ -47,7 +47,10 @@ typedef enum {
     STRATA_ERR_UNSUPPORTED = 2,  /* a shape or format outside the supported set */
     STRATA_ERR_OOM = 3,          /* device allocation failed (nothing leaked) */
     STRATA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
-    STRATA_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (see sync_status) */
+    STRATA_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out (see sync_status) */
+    STRATA_ERR_BOUNDS = 6        /* checked build (-DSTRATA_CHECKS=1) only: a device-side
+                                    gather/scatter index fell outside its buffer; the access
+                                    was skipped and reported, never faulted on */
 } strata_status;
 
 typedef struct strata_moe *strata_moe_t; /* opaque, library-owned */
@@ -171,6 +174,74 @@ const char *strata_moe_last_error(void);
  * [nrows][cols].  Synchronous. */
 strata_status strata_moe_debug_dequant(strata_moe_t h, int expert, int mat, int row0, int nrows,
                                        int kind, float *out_host);
+
+/* ---- Expert parallelism (experts of a layer split across ranks).
+ * Rank r of N owns experts [e_begin, e_end) = [ceil(r E / N), ceil((r+1) E / N)),
+ * i.e. expert e belongs to rank floor(e N / E); every rank keeps the router and
+ * the shared expert.  One forward of a rank's T tokens (the Python layer
+ * quantized_expert_ffn_04_b200.ep does this with torch.distributed
+ * all-to-alls): route -> strata_ep_plan -> send each pick's token row and
+ * expert id to the owner -> the owner runs strata_moe_expert_rows on what it
+ * got -> outputs back in the same order -> strata_moe_combine_rows.  Each
+ * expert output depends on one token row and one expert only, so the result
+ * equals the one-GPU forward bit for bit (prefill = T > 64, as there). */
+strata_status strata_ep_expert_range(int rank, int n_ranks, int n_experts, int32_t *e_begin,
+                                     int32_t *e_end);
+
+/* Host only.  idx: int32 [T][k] picks (host).  Out (host, caller-owned):
+ * send_counts [n_ranks] picks per destination rank; send_pick [T*k] the pick
+ * index t*k+j of each row to send, grouped by destination rank, inside a rank
+ * by expert id, then token (a stable, deterministic order); slot [T*k] the
+ * position of pick t*k+j in that order.  INVALID_ARG on an id outside
+ * [0, n_experts) or a bad size; nothing else can fail. */
+strata_status strata_ep_plan(const int32_t *idx, int T, int k, int n_experts, int n_ranks,
+                             int32_t *send_counts, int32_t *send_pick, int32_t *slot);
+
+/* dst row i = src row rows[i] (device buffers, rows int32 [n]); row_bytes a
+ * multiple of 16 and both buffers 16-byte aligned, else INVALID_ARG.  A row
+ * index outside [0, n_src) is skipped.  Enqueued on `stream`. */
+strata_status strata_ep_gather_rows(const void *src_dev, const int32_t *rows_dev, int n,
+                                    int n_src, int row_bytes, void *dst_dev, void *stream);
+
+/* Expert outputs of single rows: row i of x_dev (bf16 [n][H], device) goes
+ * through expert ids_dev[i] (int32 [n], device; -1: none) and, for
+ * i < n_shared, through the shared expert as well.
+ *   y_dev        [n][H] out: row i = expert ids[i](x_i) (rows with id -1 untouched)
+ *   yshared_dev  [n_shared][H] out: shared(x_i), or NULL when n_shared == 0
+ * Outputs are in the row's prescaled units (times 2^-2e, e the row's token
+ * prescale exponent), fp32 when prefill == 0 (the decode kernels) and fp16
+ * when prefill != 0 (the tensor-core kernels): exactly the values the
+ * one-GPU forward feeds its combine.  n <= max_tokens.  Enqueued on `stream`. */
+strata_status strata_moe_expert_rows(strata_moe_t h, const void *x_dev, const int32_t *ids_dev,
+                                     int n, int n_shared, int prefill, void *y_dev,
+                                     void *yshared_dev, void *stream);
+
+/* The layer's combine from expert outputs: out_t = shared + sum over the k
+ * picks in ascending expert id of w_j * Y_j, times 2^2e (the token's
+ * prescale, recomputed from x_dev), one rounding to bf16.
+ *   x_dev   bf16 [T][H] the layer input (device)
+ *   idx_dev int32 [T][k], w_dev float [T][k] the routing (device)
+ *   slot_dev int32 [T][k]: row of y_dev holding pick (t, j)
+ *   y_dev   [T*k + T][H] expert outputs, the shared expert's at row T*k + t;
+ *           fp32 (prefill == 0) or fp16 (prefill != 0), as strata_moe_expert_rows
+ *   out_dev bf16 [T][H] out.  Enqueued on `stream`. */
+strata_status strata_moe_combine_rows(strata_moe_t h, const void *x_dev, int T,
+                                      const int32_t *idx_dev, const float *w_dev,
+                                      const int32_t *slot_dev, const void *y_dev, int prefill,
+                                      void *out_dev, void *stream);
+
+/* Test hooks for the out-of-memory paths.  Every device and pinned host
+ * allocation of the library goes through one counter.
+ * strata_moe_debug_fail_alloc(n), n >= 0: the n-th allocation from now (0 =
+ * the next one) fails as if the device were out of memory, without
+ * allocating; n = -1 switches the injection off.  Process-wide, not
+ * thread-safe against concurrent creates; returns INVALID_ARG for n < -1.
+ * strata_moe_debug_live_allocs(): the number of blocks the library holds now
+ * (every handle's weights, workspace and pinned error word, plus any
+ * transient staging buffer).  A create that fails returns with this number
+ * unchanged and *out = NULL. */
+strata_status strata_moe_debug_fail_alloc(int64_t n);
+int64_t strata_moe_debug_live_allocs(void);
 
 /* Options (strata_moe_set_option). */
 enum {

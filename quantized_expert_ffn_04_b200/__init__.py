@@ -12,7 +12,10 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstrata_moe.so")
+# STRATA_MOE_CHECKED=1 loads the checked build instead (every device-side
+# gather/scatter index tested; a bad one reports STRATA_ERR_BOUNDS)
+LIB_PATH = os.path.join(_HERE, "libstrata_moe_checked.so" if os.environ.get("STRATA_MOE_CHECKED") == "1"
+                        else "libstrata_moe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -22,7 +25,7 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 STRATA_OK, STRATA_ERR_INVALID_ARG, STRATA_ERR_UNSUPPORTED, STRATA_ERR_OOM, STRATA_ERR_CUDA, \
-    STRATA_ERR_TIMEOUT = range(6)
+    STRATA_ERR_TIMEOUT, STRATA_ERR_BOUNDS = range(7)
 STRATA_OPT_PATH, STRATA_OPT_WAIT_BUDGET, STRATA_OPT_DECODE_MAX_T = 1, 2, 3
 
 # every symbol the header declares
@@ -30,7 +33,10 @@ SYMBOLS = ("strata_moe_create", "strata_moe_destroy", "strata_moe_route", "strat
            "strata_moe_forward_host", "strata_moe_rmsnorm", "strata_moe_stack_forward",
            "strata_moe_sync_status", "strata_moe_last_error", "strata_moe_debug_dequant",
            "strata_moe_set_option", "strata_moe_selftest_wait", "strata_moe_version",
-           "strata_moe_set_probe", "strata_moe_launch_count", "strata_moe_route_noalloc")
+           "strata_moe_set_probe", "strata_moe_launch_count", "strata_moe_route_noalloc",
+           "strata_moe_debug_fail_alloc", "strata_moe_debug_live_allocs",
+           "strata_ep_expert_range", "strata_ep_plan", "strata_ep_gather_rows",
+           "strata_moe_expert_rows", "strata_moe_combine_rows")
 
 
 class strata_moe_config(C.Structure):
@@ -67,6 +73,12 @@ _sig = {
     "strata_moe_set_probe": [_P, _I, _P, _P],
     "strata_moe_launch_count": [_P, _I],
     "strata_moe_route_noalloc": [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P],
+    "strata_moe_debug_fail_alloc": [_I64],
+    "strata_ep_expert_range": [_I, _I, _I, _P, _P],
+    "strata_ep_plan": [_P, _I, _I, _I, _I, _P, _P, _P],
+    "strata_ep_gather_rows": [_P, _P, _I, _I, _I, _P, _P],
+    "strata_moe_expert_rows": [_P, _P, _P, _I, _I, _I, _P, _P, _P],
+    "strata_moe_combine_rows": [_P, _P, _I, _P, _P, _P, _P, _I, _P, _P],
 }
 for _name, _args in _sig.items():
     _f = getattr(_lib, _name)
@@ -76,6 +88,8 @@ _lib.strata_moe_destroy.argtypes = [_P]
 _lib.strata_moe_destroy.restype = None
 _lib.strata_moe_last_error.restype = C.c_char_p
 _lib.strata_moe_version.restype = C.c_char_p
+_lib.strata_moe_debug_live_allocs.argtypes = []
+_lib.strata_moe_debug_live_allocs.restype = C.c_int64
 
 
 def _check(status: int):
@@ -133,6 +147,46 @@ def strata_moe_debug_dequant(h, expert, mat, row0, nrows, kind, out_host) -> Non
 
 def strata_moe_set_option(h, option, value) -> None:
     _check(_lib.strata_moe_set_option(h, option, int(value)))
+
+
+def strata_ep_expert_range(rank, n_ranks, n_experts) -> tuple[int, int]:
+    b, e = C.c_int32(), C.c_int32()
+    _check(_lib.strata_ep_expert_range(rank, n_ranks, n_experts, C.byref(b), C.byref(e)))
+    return b.value, e.value
+
+
+def strata_ep_plan(idx, n_experts, n_ranks):
+    """idx: int32 numpy [T][k] (host).  Returns (send_counts [n_ranks],
+    send_pick [T*k], slot [T*k]) as int32 numpy arrays."""
+    import numpy as np
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    counts = np.zeros(n_ranks, dtype=np.int32)
+    pick = np.zeros(T * k, dtype=np.int32)
+    slot = np.zeros(T * k, dtype=np.int32)
+    _check(_lib.strata_ep_plan(idx.ctypes.data, T, k, n_experts, n_ranks, counts.ctypes.data,
+                               pick.ctypes.data, slot.ctypes.data))
+    return counts, pick, slot
+
+
+def strata_ep_gather_rows(src, rows, n, n_src, row_bytes, dst, stream=None) -> None:
+    _check(_lib.strata_ep_gather_rows(src, rows, n, n_src, row_bytes, dst, stream))
+
+
+def strata_moe_expert_rows(h, x, ids, n, n_shared, prefill, y, yshared, stream=None) -> None:
+    _check(_lib.strata_moe_expert_rows(h, x, ids, n, n_shared, int(prefill), y, yshared, stream))
+
+
+def strata_moe_combine_rows(h, x, T, idx, w, slot, y, prefill, out, stream=None) -> None:
+    _check(_lib.strata_moe_combine_rows(h, x, T, idx, w, slot, y, int(prefill), out, stream))
+
+
+def strata_moe_debug_fail_alloc(n) -> None:
+    _check(_lib.strata_moe_debug_fail_alloc(int(n)))
+
+
+def strata_moe_debug_live_allocs() -> int:
+    return int(_lib.strata_moe_debug_live_allocs())
 
 
 def strata_moe_selftest_wait(device, budget_cycles) -> None:

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <string>
 #include <vector>
@@ -54,6 +55,61 @@ struct DeviceGuard {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---- every allocation of the library goes through these wrappers: they
+// count the live blocks and can be told to fail the n-th allocation from now
+// (a host-side fault injector for the out-of-memory paths; it never touches
+// the device beyond refusing to allocate).
+std::atomic<long long> g_alloc_seq{0};   // allocations attempted so far
+std::atomic<long long> g_fail_at{-1};    // sequence number that fails, -1: none
+std::atomic<long long> g_live{0};        // device + pinned blocks alive
+
+bool injected_failure() {
+    const long long seq = g_alloc_seq.fetch_add(1);
+    return g_fail_at.load() == seq;
+}
+cudaError_t dev_malloc(void **p, size_t n) {
+    *p = nullptr;
+    if (injected_failure()) return cudaErrorMemoryAllocation;
+    const cudaError_t e = cudaMalloc(p, n);
+    if (e != cudaSuccess) {
+        *p = nullptr;
+        cudaGetLastError();  // the failure is reported, not left sticky
+        return e;
+    }
+    if (*p) g_live.fetch_add(1);
+    return cudaSuccess;
+}
+template <class T>
+cudaError_t dev_malloc(T **p, size_t n) {
+    void *v = nullptr;
+    const cudaError_t e = dev_malloc(&v, n);
+    *p = static_cast<T *>(v);
+    return e;
+}
+void dev_free(void *p) {
+    if (!p) return;
+    cudaFree(p);
+    g_live.fetch_sub(1);
+}
+cudaError_t pinned_malloc(int **p) {
+    *p = nullptr;
+    if (injected_failure()) return cudaErrorMemoryAllocation;
+    void *v = nullptr;
+    const cudaError_t e = cudaMallocHost(&v, sizeof(int));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e;
+    }
+    *p = static_cast<int *>(v);
+    g_live.fetch_add(1);
+    return cudaSuccess;
+}
+void pinned_free(int *p) {
+    if (!p) return;
+    cudaFreeHost(p);
+    g_live.fetch_sub(1);
+}
+
 constexpr long long kDefaultBudget = 4000000000ll;  // ~2 s at the top SM clock
 
 }  // namespace
@@ -68,6 +124,9 @@ struct strata_moe {
     __half *router_split = nullptr;  // [router_rows][H]: fp16(W) rows, then fp16(W - fp16(W))
     int router_rows = 0;             // 2E rounded up to 128
     float screen_gam = 0.f, screen_wmax = 0.f, screen_bmax = 0.f;
+    // token prescale bound: the largest gate/up row L2 norm times
+    // sqrt(max(1, sqrt(I) * (largest down row L2 norm) / 2)), padded 0.1 %
+    float w2eff = 0.f;
     void *ws = nullptr;
     size_t ws_bytes = 0;
     // workspace views
@@ -93,6 +152,7 @@ struct strata_moe {
     int *fused_cnt = nullptr;
     int fused_stride = 0, fused_tok = 0;
     int *xex = nullptr;
+    int *slot_ex = nullptr;       // [slots] prefill: the token exponent of every slot
     float *fcorr = nullptr;  // [min(max_tokens, 64)][H / 32] block corrections of the fused layer
     cudaEvent_t probe_begin[6] = {}, probe_end[6] = {};
     // options
@@ -181,18 +241,19 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->fused_bar = (unsigned long long *)take(8);
     h->fused_cnt = (int *)take((size_t)2 * h->fused_stride * 4);
     h->xex = (int *)take(T * 4);
+    h->slot_ex = (int *)take(slots * 4);
     h->fcorr = (float *)take((T < 64 ? T : 64) * (H / 32) * 4);
     return off;
 }
 
 void free_handle(strata_moe *h) {
     if (!h) return;
-    cudaFree(h->wq);
-    cudaFree(h->router_wp);
-    cudaFree(h->router_b);
-    cudaFree(h->router_split);
-    cudaFree(h->ws);
-    if (h->err_host) cudaFreeHost(h->err_host);
+    dev_free(h->wq);
+    dev_free(h->router_wp);
+    dev_free(h->router_b);
+    dev_free(h->router_split);
+    dev_free(h->ws);
+    pinned_free(h->err_host);
     delete h;
 }
 
@@ -257,13 +318,13 @@ strata_status run_route(strata_moe_t h, const void *x, int T, int tile, cudaStre
     if (T > kSmallMaxT) {
         probe(h, kStDispatch, true, s);
         launch_dispatch(h->idx, T, g.k, g.E, h->cnt, h->off, h->list, h->slot, h->ds, h->units,
-                        h->n_units, tile, s);
+                        h->n_units, tile, s, h->err);
         probe(h, kStDispatch, false, s);
     } else {
         // top-k and dispatch fused in one CTA (the top-k probe brackets both)
         probe(h, kStTopk, true, s);
         launch_route_small(h->logits, T, g.E, g.k, h->idx, h->wts, h->cnt, h->off, h->list,
-                           h->slot, h->units, h->n_units, tile, s);
+                           h->slot, h->units, h->n_units, tile, s, h->err);
         probe(h, kStTopk, false, s);
     }
     return check_launch("routing kernels");
@@ -293,7 +354,7 @@ strata_status run_forward_fused(strata_moe_t h, const void *x, int T, void *y, b
     fa.x = x;
     fa.router_wp = h->router_wp;
     fa.router_b = h->router_b;
-    fa.w2 = 0.0f;
+    fa.w2 = h->w2eff;
     fa.logits = h->logits;
     fa.idx = h->idx;
     fa.wts = h->wts;
@@ -324,14 +385,17 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
     const Geometry &g = h->geo;
     const bool decode = use_decode_path(h, T);
     const int tile = decode ? 8 : kUmmaTile;
+    // the decode chain's token exponents: a plain launch ahead of the router,
+    // so every later kernel starts after it completed
+    if (decode) launch_prescale(x, T, g.H, h->w2eff, h->xex, nullptr, s);
     strata_status st = run_route(h, x, T, tile, s);
     if (st != STRATA_OK) return st;
     ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
     int umax = max_units(T, g.k, g.E, tile);
     if (decode) {
         probe(h, kStGateUp, true, s);
-        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, T, x, h->a,
-                           h->err, h->budget, s);
+        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, T * g.k, T, x, h->xex,
+                           h->a, h->err, h->budget, s);
         probe(h, kStGateUp, false, s);
         probe(h, kStDown, true, s);
         launch_gemv_down(g, w, h->units, h->n_units, umax, T, h->a, (float *)h->Y, h->err,
@@ -341,10 +405,13 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
         // the gate/up probe brackets the gate/up GEMM (and, for T <= kSmallMaxT,
         // the fp16 token copy, which larger batches make in the router stage)
         probe(h, kStGateUp, true, s);
-        if (T <= kSmallMaxT) launch_to_half(x, x16_of(h, T), (size_t)T * g.H, s);
-        launch_gather_rows(h->list, T * g.k, x16_of(h, T), h->xs, g.H, s);
+        // the prescaled fp16 token operand (above kSmallMaxT it replaces the
+        // unscaled copy the router's screening GEMM read)
+        launch_prescale(x, T, g.H, h->w2eff, h->xex, x16_of(h, T), s);
+        launch_gather_rows(h->list, T * g.k, x16_of(h, T), h->xs, g.H, s, T, h->err, h->xex,
+                           h->slot_ex);
         cudaError_t ce = launch_umma_gateup(g, w, h->units, h->n_units, umax, T * g.k + T, h->xs,
-                                            h->a, h->err, h->budget, s);
+                                            h->slot_ex, h->a, h->err, h->budget, s);
         if (ce != cudaSuccess)
             return fail(STRATA_ERR_CUDA, "gate/up GEMM: %s", cudaGetErrorString(ce));
         probe(h, kStGateUp, false, s);
@@ -356,7 +423,8 @@ strata_status run_forward(strata_moe_t h, const void *x, int T, void *y, bool re
         probe(h, kStDown, false, s);
     }
     probe(h, kStCombine, true, s);
-    launch_combine(h->Y, !decode, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s);
+    launch_combine(h->Y, !decode, h->idx, h->wts, h->slot, T, g.k, g.H, y, residual, s, h->err,
+                   h->xex);
     probe(h, kStCombine, false, s);
     return check_launch("expert kernels");
 }
@@ -383,13 +451,13 @@ int strata_moe_launch_count(strata_moe_t h, int T) {
     if (!h || T < 0 || T > h->cfg.max_tokens) return 0;
     if (T == 0) return 0;
     // up to kSmallMaxT tokens: router, fused top-k + dispatch; above: fp16 token
-    // copy, screening GEMM, screened top-k, 3 dispatch kernels.  Then gate/up +
-    // down (the tensor-core path adds the slot-order row gather, and the fp16
-    // token copy when T <= kSmallMaxT), and the combine.
+    // copy, screening GEMM, screened top-k, 3 dispatch kernels.  Then the token
+    // prescale, gate/up + down (the tensor-core path adds the slot-order row
+    // gather), and the combine.
     if (use_fused_path(h, T)) return 1;  // the fused layer kernel
     const bool decode = use_decode_path(h, T);
-    if (T <= kSmallMaxT) return 2 + (decode ? 2 : 4) + 1;
-    return 6 + 3 + 1;
+    if (T <= kSmallMaxT) return 2 + 1 + (decode ? 2 : 3) + 1;
+    return 6 + 1 + 3 + 1;
 }
 
 strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_weights *wts,
@@ -421,11 +489,10 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
 
     // ---- allocations
     size_t ws_bytes = carve_workspace(h, nullptr);
-    if (cudaMalloc(&h->wq, (E + 1) * g.expert_bytes) != cudaSuccess ||
-        cudaMalloc(&h->router_wp, E * H * 4) != cudaSuccess ||
-        (cfg->has_router_bias && cudaMalloc(&h->router_b, E * 4) != cudaSuccess) ||
-        cudaMalloc(&h->ws, ws_bytes) != cudaSuccess) {
-        cudaGetLastError();
+    if (dev_malloc(&h->wq, (E + 1) * g.expert_bytes) != cudaSuccess ||
+        dev_malloc(&h->router_wp, E * H * 4) != cudaSuccess ||
+        (cfg->has_router_bias && dev_malloc(&h->router_b, E * 4) != cudaSuccess) ||
+        dev_malloc(&h->ws, ws_bytes) != cudaSuccess) {
         size_t wbytes = (E + 1) * g.expert_bytes;
         free_handle(h);
         return fail(STRATA_ERR_OOM, "device allocation failed (weights %zu B, workspace %zu B)",
@@ -433,10 +500,9 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
     }
     h->ws_bytes = ws_bytes;
     carve_workspace(h, (char *)h->ws);
-    if ((ce = cudaMallocHost(&h->err_host, 4)) != cudaSuccess) {
-        h->err_host = nullptr;
+    if (pinned_malloc(&h->err_host) != cudaSuccess) {
         free_handle(h);
-        return cuda_fail(ce, "cudaMallocHost(error word)");
+        return fail(STRATA_ERR_OOM, "pinned host allocation (error word) failed");
     }
     *h->err_host = 0;
     if ((ce = cudaMemset(h->ws, 0, ws_bytes)) != cudaSuccess) {
@@ -474,8 +540,7 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
         h->screen_gam = (float)(H * std::ldexp(1.0, -23) + std::ldexp(1.0, -22) +
                                 (H / 32.0 + 10.0) * std::ldexp(1.0, -24));
         if (ce == cudaSuccess) {
-            if (cudaMalloc(&h->router_split, R * H * 2) != cudaSuccess) {
-                cudaGetLastError();
+            if (dev_malloc(&h->router_split, R * H * 2) != cudaSuccess) {
                 free_handle(h);
                 return fail(STRATA_ERR_OOM, "router split allocation failed");
             }
@@ -496,13 +561,16 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
         const size_t batch = 32;
         uint8_t *tc = nullptr;
         uint16_t *ts = nullptr;
-        if (cudaMalloc(&tc, batch * ex_codes) != cudaSuccess ||
-            cudaMalloc(&ts, batch * ex_scales * 2) != cudaSuccess) {
-            cudaGetLastError();
-            cudaFree(tc);
+        unsigned *nrm = nullptr;  // [0] gate/up rows, [1] down rows: largest L2 norm (float bits)
+        if (dev_malloc(&tc, batch * ex_codes) != cudaSuccess ||
+            dev_malloc(&ts, batch * ex_scales * 2) != cudaSuccess ||
+            dev_malloc(&nrm, 2 * sizeof(unsigned)) != cudaSuccess) {
+            dev_free(tc);
+            dev_free(ts);
             free_handle(h);
             return fail(STRATA_ERR_OOM, "staging allocation failed");
         }
+        ce = cudaMemset(nrm, 0, 2 * sizeof(unsigned));
         for (size_t e0 = 0; e0 <= E && ce == cudaSuccess; e0 += batch) {
             size_t nb = (E + 1 - e0) < batch ? (E + 1 - e0) : batch;  // expert E = shared
             for (size_t i = 0; i < nb && ce == cudaSuccess; i++) {
@@ -519,23 +587,34 @@ strata_status strata_moe_create(const strata_moe_config *cfg, const strata_moe_w
                 for (int m = 0; m < 3; m++) {
                     const uint8_t *c = tc + i * ex_codes + m * mat_codes;
                     const uint16_t *s = ts + i * ex_scales + m * mat_scales;
-                    if (m < 2)
+                    if (m < 2) {
                         launch_repack_matrix(c, s, g.bits, g.I, g.H, g.Ip, g.H,
                                              dst + m * g.mat_bytes, 0);
-                    else
+                        launch_row_norm_max(c, s, g.bits, g.I, g.H, nrm, 0);
+                    } else {
                         launch_repack_matrix(c, s, g.bits, g.H, g.I, g.H, g.Ip,
                                              dst + m * g.mat_bytes, 0);
+                        launch_row_norm_max(c, s, g.bits, g.H, g.I, nrm + 1, 0);
+                    }
                 }
                 ce = cudaGetLastError();
             }
             if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
         }
-        cudaFree(tc);
-        cudaFree(ts);
+        unsigned nb[2] = {0u, 0u};
+        if (ce == cudaSuccess) ce = cudaMemcpy(nb, nrm, sizeof nb, cudaMemcpyDeviceToHost);
+        dev_free(tc);
+        dev_free(ts);
+        dev_free(nrm);
         if (ce != cudaSuccess) {
             free_handle(h);
             return cuda_fail(ce, "expert upload / repack");
         }
+        float w2, wd2;
+        memcpy(&w2, &nb[0], 4);
+        memcpy(&wd2, &nb[1], 4);
+        const double c = std::max(1.0, std::sqrt((double)g.I) * wd2 / 2.0);
+        h->w2eff = (float)(w2 * std::sqrt(c) * 1.001);
     }
     *out = h;
     return STRATA_OK;
@@ -627,6 +706,8 @@ strata_status strata_moe_sync_status(strata_moe_t h, void *stream) {
         cudaMemsetAsync(h->fused_bar, 0, 8, s);
         cudaMemsetAsync(h->fused_cnt, 0, (size_t)2 * h->fused_stride * 4, s);
         cudaStreamSynchronize(s);
+        if (e == kErrBounds)
+            return fail(STRATA_ERR_BOUNDS, "a device-side index check failed (checked build)");
         return fail(STRATA_ERR_TIMEOUT, "a device-side wait gave up (code %d)", e);
     }
     return STRATA_OK;
@@ -717,12 +798,12 @@ strata_status strata_moe_debug_dequant(strata_moe_t h, int expert, int mat, int 
     const uint8_t *m = h->wq + e * g.expert_bytes + mat * g.mat_bytes;
     float *d = nullptr;
     size_t n = (size_t)nrows * cols;
-    cudaError_t ce = cudaMalloc(&d, n * 4);
+    cudaError_t ce = dev_malloc(&d, n * 4);
     if (ce != cudaSuccess) return fail(STRATA_ERR_OOM, "debug buffer");
     launch_debug_dequant(m, g.bits, Kp, row0, nrows, cols, kind, d, 0);
     ce = cudaGetLastError();
     if (ce == cudaSuccess) ce = cudaMemcpy(out_host, d, n * 4, cudaMemcpyDeviceToHost);
-    cudaFree(d);
+    dev_free(d);
     if (ce != cudaSuccess) return cuda_fail(ce, "debug dequant");
     return STRATA_OK;
 }
@@ -734,16 +815,90 @@ strata_status strata_moe_selftest_wait(int device, int64_t budget_cycles) {
     if (device < 0 || device >= ndev) return fail(STRATA_ERR_INVALID_ARG, "bad device");
     DeviceGuard guard(device);
     int *err = nullptr;
-    if (cudaMalloc(&err, 4) != cudaSuccess) return fail(STRATA_ERR_OOM, "selftest buffer");
+    if (dev_malloc(&err, 4) != cudaSuccess) return fail(STRATA_ERR_OOM, "selftest buffer");
     cudaMemset(err, 0, 4);
     launch_selftest_wait(err, budget_cycles, 0);
     int e = 0;
     ce = cudaGetLastError();
     if (ce == cudaSuccess) ce = cudaMemcpy(&e, err, 4, cudaMemcpyDeviceToHost);
-    cudaFree(err);
+    dev_free(err);
     if (ce != cudaSuccess) return cuda_fail(ce, "selftest");
     if (e) return fail(STRATA_ERR_TIMEOUT, "the bounded wait gave up as designed");
     return STRATA_OK;
 }
+
+strata_status strata_moe_expert_rows(strata_moe_t h, const void *x_dev, const int32_t *ids_dev,
+                                     int n, int n_shared, int prefill, void *y_dev,
+                                     void *yshared_dev, void *stream) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    if (n < 0 || n > h->cfg.max_tokens || n_shared < 0 || n_shared > n)
+        return fail(STRATA_ERR_INVALID_ARG, "n=%d / n_shared=%d out of range (max_tokens %d)", n,
+                    n_shared, h->cfg.max_tokens);
+    if (n == 0) return STRATA_OK;
+    if (!x_dev || !ids_dev || !y_dev || (n_shared > 0 && !yshared_dev))
+        return fail(STRATA_ERR_INVALID_ARG, "NULL buffer");
+    DeviceGuard guard(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Geometry &g = h->geo;
+    const int tile = prefill ? kUmmaTile : 8;
+    ExpertWeights w{h->wq, h->wq + (size_t)g.E * g.expert_bytes};
+    const int umax = max_units(n, 1, g.E, tile);
+    // rows = tokens with one routed pick each (k = 1); slots: picks in
+    // dispatch order, then the shared expert's rows at n + t
+    __half *x16 = prefill ? reinterpret_cast<__half *>(h->xs) + (size_t)n * g.H : nullptr;
+    launch_prescale(x_dev, n, g.H, h->w2eff, h->xex, x16, s);
+    launch_dispatch(ids_dev, n, 1, g.E, h->cnt, h->off, h->list, h->slot, h->ds, h->units,
+                    h->n_units, tile, s, h->err, n_shared);
+    if (!prefill) {
+        launch_gemv_gateup(g, w, h->units, h->n_units, umax, h->list, n, n, x_dev, h->xex, h->a,
+                           h->err, h->budget, s, n_shared);
+        launch_gemv_down(g, w, h->units, h->n_units, umax, n, h->a, (float *)h->Y, h->err,
+                         h->budget, s);
+    } else {
+        launch_gather_rows(h->list, n, x16, h->xs, g.H, s, n, h->err, h->xex, h->slot_ex);
+        cudaError_t ce = launch_umma_gateup(g, w, h->units, h->n_units, umax, 2 * n, h->xs,
+                                            h->slot_ex, h->a, h->err, h->budget, s);
+        if (ce == cudaSuccess)
+            ce = launch_umma_down(g, w, h->units, h->n_units, umax, 2 * n, h->a, h->Y, h->err,
+                                  h->budget, s);
+        if (ce != cudaSuccess)
+            return fail(STRATA_ERR_CUDA, "expert GEMM: %s", cudaGetErrorString(ce));
+    }
+    const int eb = prefill ? 2 : 4, rb = g.H * eb;
+    launch_gather_rows_bytes(h->Y, h->slot, n, n, rb, y_dev, h->err, s, ids_dev);
+    if (n_shared > 0) {
+        cudaError_t ce = cudaMemcpyAsync(yshared_dev, (const char *)h->Y + (size_t)n * rb,
+                                         (size_t)n_shared * rb, cudaMemcpyDeviceToDevice, s);
+        if (ce != cudaSuccess) return cuda_fail(ce, "shared rows copy");
+    }
+    return check_launch("expert rows");
+}
+
+strata_status strata_moe_combine_rows(strata_moe_t h, const void *x_dev, int T,
+                                      const int32_t *idx_dev, const float *w_dev,
+                                      const int32_t *slot_dev, const void *y_dev, int prefill,
+                                      void *out_dev, void *stream) {
+    if (!h) return fail(STRATA_ERR_INVALID_ARG, "handle is NULL");
+    strata_status st = check_tokens(h, T);
+    if (st != STRATA_OK) return st;
+    if (T == 0) return STRATA_OK;
+    if (!x_dev || !idx_dev || !w_dev || !slot_dev || !y_dev || !out_dev)
+        return fail(STRATA_ERR_INVALID_ARG, "NULL buffer");
+    DeviceGuard guard(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Geometry &g = h->geo;
+    launch_prescale(x_dev, T, g.H, h->w2eff, h->xex, nullptr, s);
+    launch_combine(y_dev, prefill != 0, idx_dev, w_dev, slot_dev, T, g.k, g.H, out_dev, false, s,
+                   h->err, h->xex);
+    return check_launch("combine rows");
+}
+
+strata_status strata_moe_debug_fail_alloc(int64_t n) {
+    if (n < -1) return fail(STRATA_ERR_INVALID_ARG, "n must be >= -1");
+    g_fail_at.store(n < 0 ? -1 : g_alloc_seq.load() + n);
+    return STRATA_OK;
+}
+
+int64_t strata_moe_debug_live_allocs(void) { return g_live.load(); }
 
 }  // extern "C"

@@ -46,7 +46,8 @@ constexpr int kCombineThreads = 64;
 template <typename YT>
 __global__ __launch_bounds__(kCombineThreads) void combine_kernel(
     const YT *__restrict__ Y, const int32_t *__restrict__ idx, const float *__restrict__ w,
-    const int32_t *__restrict__ slot, int T, int k, int H, __nv_bfloat16 *out, int residual) {
+    const int32_t *__restrict__ slot, int T, int k, int H, __nv_bfloat16 *out, int residual,
+    int *err, const int *__restrict__ xex) {
     __shared__ int re[32], rs[32], ss[32];
     __shared__ float rw[32], sw[32];
     const int t = blockIdx.x;
@@ -75,10 +76,19 @@ __global__ __launch_bounds__(kCombineThreads) void combine_kernel(
 #pragma unroll 4
     for (int i = 0; i < k; i++) {
         float v[8];
+        if (!idx_ok(err, ss[i], Tk)) continue;
         load8<YT>(Y + (size_t)ss[i] * H + c, v);
         const float wi = sw[i];
 #pragma unroll
         for (int q = 0; q < 8; q++) acc[q] = fmaf(wi, v[q], acc[q]);
+    }
+    if (xex) {  // Y in the token's prescaled units: undo 2^-2e (two steps stay in range)
+        const int e = xex[t];
+        if (e) {
+            const float f = pow2f(e);
+#pragma unroll
+            for (int q = 0; q < 8; q++) acc[q] = acc[q] * f * f;
+        }
     }
     __nv_bfloat16 *o = out + (size_t)t * H + c;
     uint4 hv = make_uint4(0, 0, 0, 0);
@@ -96,17 +106,17 @@ __global__ __launch_bounds__(kCombineThreads) void combine_kernel(
 
 void launch_combine(const void *Y, bool y_half, const int32_t *idx, const float *w,
                     const int32_t *slot, int T, int k, int H, void *out, bool residual,
-                    cudaStream_t s) {
+                    cudaStream_t s, int *err, const int *xex) {
     auto o = reinterpret_cast<__nv_bfloat16 *>(out);
     dim3 grid(T, (H + kCombineCols - 1) / kCombineCols);
     if (y_half)
         launch_pdl(combine_kernel<__half>, grid, dim3(kCombineThreads), 0, s,
                    reinterpret_cast<const __half *>(Y), idx, w, slot, T, k, H, o,
-                   residual ? 1 : 0);
+                   residual ? 1 : 0, err, xex);
     else
         launch_pdl(combine_kernel<float>, grid, dim3(kCombineThreads), 0, s,
                    reinterpret_cast<const float *>(Y), idx, w, slot, T, k, H, o,
-                   residual ? 1 : 0);
+                   residual ? 1 : 0, err, xex);
 }
 
 // ------------------------------------------------------------------ RMSNorm

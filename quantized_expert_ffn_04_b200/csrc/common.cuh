@@ -56,6 +56,25 @@ __host__ __device__ constexpr int unit_bytes(int bits) {
 // ---------------------------------------------------------------- errors
 // Device error word codes (handle workspace).
 constexpr int kErrTimeout = 1;
+constexpr int kErrBounds = 2;  // checked build: a gather/scatter index was out of range
+
+// Index check of the checked build (compiled with -DSTRATA_CHECKS=1): true
+// when 0 <= i < n; otherwise the error word (if any) gets kErrBounds and the
+// caller skips the access.  In the normal build it is constant true and
+// compiles away.  It never traps: a bad index is reported, not faulted on.
+#ifndef STRATA_CHECKS
+#define STRATA_CHECKS 0
+#endif
+__device__ __forceinline__ bool idx_ok(int *err, long long i, long long n) {
+#if STRATA_CHECKS
+    if (i >= 0 && i < n) return true;
+    if (err) atomicCAS(err, 0, kErrBounds);
+    return false;
+#else
+    (void)err, (void)i, (void)n;
+    return true;
+#endif
+}
 
 // ---------------------------------------------------------------- smem / PTX
 STRATA_DEV uint32_t smem_u32(const void *p) {
@@ -425,6 +444,72 @@ STRATA_DEV uint32_t dq2_mul(int j) {
 }
 STRATA_DEV uint32_t dq2_off(int j) {
     return j == 0 ? 0xE006E006u : j == 1 ? 0xD818D818u : j == 2 ? 0xD060D060u : 0xC980C980u;
+}
+
+// ---------------------------------------------------------- token prescale
+// The expert kernels take the token operand in fp16, whose range (largest
+// 65504, smallest normal 2^-14) is far narrower than bf16's.  Every token row
+// x is therefore scaled by an exact power of two, x' = x 2^-e, with e the
+// smallest integer such that
+//   max_i |x'_i| <= 2^9   (the 2-bit magic-offset operand x' 2^6 stays < 2^15), and
+//   ||x'||_2 w2 <= 2^7    where w2 bounds the L2 norm of every gate/up row of
+//                         the layer (times the down-row factor folded in on
+//                         the host), so by Cauchy-Schwarz |gate'|, |up'| <= 2^7,
+//                         the SwiGLU output a'' = silu(g) u 2^-2e <= 2^14 and
+//                         every down output row stays below 2^15.
+// The gate is unscaled for the sigmoid, a'' and the down outputs stay in
+// prescaled units, and the combine multiplies by 2^e twice.  Small rows get
+// e < 0 (scaled up), so their operand does not underflow.  e is clamped to
+// [-120, 120]; an all-zero or non-finite row takes e = 0.
+
+// ceil(log2 v) for finite v > 0, subnormals included.
+STRATA_DEV int ceil_log2f(float v) {
+    const int bits = __float_as_int(v), b = (bits >> 23) & 0xff, mant = bits & 0x7fffff;
+    if (b == 0) return (32 - __clz(mant - 1)) - 149;
+    return b - 127 + (mant ? 1 : 0);
+}
+STRATA_DEV float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
+
+// First step: the exponent from the row's largest magnitude m alone.
+STRATA_DEV int prescale_emax(float m) {
+    if (!(m > 0.0f) || m > 3.0e38f) return 0;
+    const int e = ceil_log2f(m) - 9;
+    return e < -120 ? -120 : (e > 120 ? 120 : e);
+}
+// Final exponent: em from prescale_emax, ss = sum over the row of (x_i 2^-em)^2
+// (in fp32: every term is at most 2^18, so no overflow), w2 the layer bound
+// (0: no bound, em alone).
+STRATA_DEV int prescale_final(int em, float ss, float w2) {
+    if (!(w2 > 0.0f)) return em;
+    const float v = sqrtf(ss) * w2 * 1.001f;
+    const int d = (v > 128.0f && v < 3.0e38f) ? ceil_log2f(v) - 7 : 0;
+    const int e = em + d;
+    return e > 120 ? 120 : e;
+}
+// The prescale exponent of one bf16 row of length H, computed by one warp in
+// one fixed order (lane l takes i = l, l + 32, ... with fma, then a halving
+// tree), so every kernel that needs it gets the same e.  All lanes return e.
+STRATA_DEV int token_prescale_warp(const __nv_bfloat16 *row, int H, float w2, int lane) {
+    float m = 0.0f;
+    for (int i = lane; i < H; i += 32) m = fmaxf(m, fabsf(__bfloat162float(row[i])));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int em = prescale_emax(m);
+    const float sc = pow2f(-em);
+    float ss = 0.0f;
+    for (int i = lane; i < H; i += 32) {
+        const float v = __bfloat162float(row[i]) * sc;
+        ss = fmaf(v, v, ss);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    return prescale_final(em, ss, w2);
+}
+// SwiGLU of a prescaled token (g, u are gate and up times 2^-ex): silu of the
+// true gate, the product left in prescaled units (times 2^-2ex).
+STRATA_DEV float swiglu_ps(float g, float u, int ex) {
+    const float gt = ex ? g * pow2f(ex) : g;
+    return g / (1.0f + expf(-gt)) * u;
 }
 
 STRATA_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {

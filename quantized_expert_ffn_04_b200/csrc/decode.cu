@@ -66,6 +66,7 @@
 namespace strata {
 
 constexpr int kFWarps = 16;                     // compute warps
+constexpr bool kFExtras = false;                // shared-expert slabs before routing
 constexpr int kGroups = 2, kGWarps = 8;         // two groups of 8 take alternate ring positions
 constexpr int kFCompute = 32 * kFWarps;         // compute threads
 constexpr int kWCopy = kFWarps, kWPub = kFWarps + 1, kWFetch = kFWarps + 2, kWComb = kFWarps + 3;
@@ -385,14 +386,6 @@ STRATA_DEV bool grid_barrier(unsigned long long *bar, unsigned long long target,
     }
 }
 
-// Smallest e >= 0 with v * 2^-e <= 2^7 (v >= 0), from the float's exponent.
-STRATA_DEV int prescale_exp(float v) {
-    const int b = (__float_as_int(v) >> 23) & 0xff;     // biased exponent
-    if (b == 0) return 0;                                // zero / subnormal
-    const int e = b - 127 + ((__float_as_int(v) & 0x7fffff) ? 1 : 0);  // ceil(log2 v)
-    return e > 7 ? e - 7 : 0;
-}
-STRATA_DEV float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
 
 // The expert token operand of column i of a token row, and the block
 // correction of the magic-offset form (2-bit): B_i = fp16(x_i 2^-ex s(i mod 32)),
@@ -412,8 +405,225 @@ STRATA_DEV float block_correction(const __nv_bfloat16 *blk, int ex) {
     return v;
 }
 
+
+// The ring items of one compute warp: its group's positions jpos, jpos + 2,
+// ... up to `stop`.  Returns the next position, or -1 once the end marker is
+// seen or the launch aborts.  One non-inlined copy serves both calls (the
+// shared expert's slabs before routing, then the routed items), so the hot
+// loop exists once per kernel instantiation and stays in the instruction
+// caches next to the other roles' loops.
+//   gate/up slab: warp q of the group takes an eighth of K of both the gate
+//   and the up slab; down block: warp q the slabs 2 (q >> 1), 2 (q >> 1) + 1,
+//   half of K; the last of the group's 8 warps to finish an item completes it.
 template <int kBits, bool kStaged>
-__global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedParams p) {
+__device__ __noinline__ int fused_run_items(const FusedParams &p, int jpos, int stop) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    constexpr int UB = unit_bytes(kBits);
+    constexpr bool kMagic = kBits == 2;
+    constexpr bool staged = kStaged;
+    const FusedSmem L = fused_smem(p.T, p.E, p.k, p.H, p.Ip, p.ring, p.item_bytes, p.staged,
+                                   p.units_max, p.na);
+    uint8_t *ring = sm + L.ring;
+    float *red = reinterpret_cast<float *>(sm + L.red);
+    __half *xs = reinterpret_cast<__half *>(sm + L.xs);
+    float *scorr = reinterpret_cast<float *>(sm + L.corr);
+    __half *abuf0 = reinterpret_cast<__half *>(sm + L.rega);
+    int4 *units = reinterpret_cast<int4 *>(sm + L.units);
+    int *slist = reinterpret_cast<int *>(sm + L.slist);
+    int *sex = reinterpret_cast<int *>(sm + L.sex);
+    int *misc = reinterpret_cast<int *>(sm + L.misc);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + L.bars);
+    uint64_t *empty = full + kFMaxRing;
+    uint64_t *abar = empty + kFMaxRing + 8;
+    uint64_t *aempty = abar + kMaxA;
+    volatile int *abort_flag = misc + kMiscAbort;
+    volatile int *vmisc = misc;
+    const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) % kGWarps;
+    const int g = lane >> 2, cq = lane & 3;
+    const int T = p.T, H = p.H, Tk = T * p.k;
+    const int nbh = H / 32, nbi = p.Ip / 32;
+    const int nsl = p.Ip / kSlabRows;              // gate/up slabs per unit
+    const int ndn = H / (kSlabRows * kDownSlabs);  // down blocks per unit
+    const int nsh = (T + kFTile - 1) / kFTile;     // shared-expert units
+    const size_t gu_bytes = (size_t)p.nseg_h * UB;
+
+auto slot_exp = [&](int sl) -> int {  // the prescale exponent of a slot's token
+    const int t = sl < Tk ? slist[sl] : sl - Tk;
+    return staged ? sex[t] : __ldcg(p.xex + t);
+};
+auto slot_tok = [&](int sl) -> int { return sl < Tk ? slist[sl] : sl - Tk; };
+// count this warp in for the item in `slot`; true for the last of the group
+auto last_warp = [&](int slot) -> bool {
+    int old = 0;
+    if (lane == 0) {
+        __threadfence_block();
+        old = atomicAdd(misc + kMiscGCnt + slot, 1);
+        if (old == kGWarps - 1) {
+            misc[kMiscGCnt + slot] = 0;  // before the slot can be refilled
+            __threadfence_block();
+        }
+    }
+    const bool last = __shfl_sync(0xffffffffu, old, 0) == kGWarps - 1;
+    __syncwarp();
+    return last;
+};
+    for (; jpos < stop; jpos += kGroups) {
+        const int slot = jpos % p.ring;
+        if (!warp_fwait(&full[slot], (jpos / p.ring) & 1, p, abort_flag, lane)) return -1;
+        const int meta = vmisc[kMiscMeta + slot];
+        if (meta == kItemEnd) return -1;
+        const int kind = item_kind(meta);
+        int u, part, slot0, n;
+        if (kind == kKindExtra) {
+            const int i = meta & 0xfffffff;
+            u = i / nsl;
+            part = i % nsl;
+            slot0 = Tk + u * kFTile;
+            n = T - u * kFTile < kFTile ? T - u * kFTile : kFTile;
+        } else {
+            const int ug0 = kFExtras && staged ? nsh : 0;
+            if (kind == kKindGU) {
+                const int it = meta & 0xfffffff;
+                u = ug0 + it / nsl;
+                part = it % nsl;
+            } else {
+                const int d = meta & 0xfffff;
+                u = d / ndn;
+                part = d % ndn;
+            }
+            const int4 un = units[u];
+            slot0 = un.y;
+            n = un.z;
+        }
+        const uint8_t *w = ring + (size_t)slot * p.item_bytes;
+        float *rd = red + (size_t)slot * (kRedSlot / 4);  // [warp of group][lane][8]
+        float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+        if (kind != kKindDown) {
+            // ---------------------------------- gate/up slab, K eighth q
+            // pairs of blocks: every range starts at an even block
+            const int b0 = 2 * (q * (nbh / 2) / 8), b1 = 2 * ((q + 1) * (nbh / 2) / 8);
+            // the lane's two token columns (columns past n repeat token 0)
+            const int ta = slot_tok(slot0 + (2 * cq < n ? 2 * cq : 0));
+            const int tb = slot_tok(slot0 + (2 * cq + 1 < n ? 2 * cq + 1 : 0));
+            if constexpr (kStaged) {
+                const int r = lane & 7;
+                const __half *rowp = xs + (size_t)slot_tok(slot0 + (r < n ? r : 0)) * (H + 8);
+                slab2_blocks<kBits, kSrcSmem, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
+                                                      scorr + ta * nbh, scorr + tb * nbh, lane);
+            } else {
+                const __half *rowp = p.x16 + (size_t)slot_tok(slot0 + (g < n ? g : 0)) * H;
+                slab2_blocks<kBits, kSrcLdg, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
+                                                     p.corr + (size_t)ta * nbh,
+                                                     p.corr + (size_t)tb * nbh, lane);
+            }
+            float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
+            rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+            rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
+            __syncwarp();
+            if (!last_warp(slot)) {
+                if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
+                continue;
+            }
+            // the last warp: the K eighths in a fixed order, then SwiGLU
+            float gs[4] = {0.f, 0.f, 0.f, 0.f}, us[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < kGWarps; j++) {
+                const float4 *rj = reinterpret_cast<const float4 *>(rd + ((size_t)j * 32 + lane) * 8);
+                const float4 vg = rj[0], vu = rj[1];
+                gs[0] += vg.x; gs[1] += vg.y; gs[2] += vg.z; gs[3] += vg.w;
+                us[0] += vu.x; us[1] += vu.y; us[2] += vu.z; us[3] += vu.w;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);  // weights and partials consumed
+            // undo the operand factor: 2^8 (magic-offset form) or 2 (exact integers)
+            const float back = kMagic ? 1.0f / 256.0f : 0.5f;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int tok = 2 * cq + (i & 1);
+                const float gv = gs[i] * back, uv = us[i] * back;
+                // silu of the true gate value; the product stays in the
+                // token's prescaled units (times 2^-2ex)
+                const int ex = slot_exp(slot0 + (tok < n ? tok : 0));
+                const float av = swiglu_ps(gv, uv, ex);
+                const int row = part * kSlabRows + g + 8 * (i >> 1);
+                if (tok < n) p.a[(size_t)(slot0 + tok) * p.Ip + row] = __float2half_rn(av);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                // post the slab's unit for the publish warp (CTA scope)
+                __threadfence_block();
+                const int idx = atomicAdd(misc + kMiscPubN, 1);
+                long long t0 = clock64();
+                while (idx - vmisc[kMiscPubSeen] >= kPubQ) {
+                    if (*abort_flag || clock64() - t0 > p.budget) {
+                        atomicCAS(p.err, 0, kErrTimeout);
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+                vmisc[kMiscPubQ + idx % kPubQ] = u + 1;
+            }
+        } else {
+            // ------------------ down block: slabs 2 (q >> 1) + {0, 1}, K half q & 1
+            const int kd = (meta >> 20) & 0xff, b = kd % p.na;
+            if (!warp_fwait(&abar[b], (kd / p.na) & 1, p, abort_flag, lane)) return -1;
+            const __half *abuf = abuf0 + (size_t)b * kFTile * (p.Ip + 8);
+            const int ar = lane & 7, pr = q >> 1, h = q & 1;
+            const __half *rowp = abuf + (size_t)(ar < n ? ar : 0) * (p.Ip + 8);
+            const uint8_t *s0 = w + (size_t)(2 * pr) * p.nseg_i * UB;
+            slab2_blocks<kBits, kSrcSmem, false>(a0, a1, s0, s0 + (size_t)p.nseg_i * UB,
+                                                 2 * (h * (nbi / 2) / 2), 2 * ((h + 1) * (nbi / 2) / 2), rowp, nullptr,
+                                                 nullptr, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&aempty[b]);  // activation rows consumed
+            float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
+            rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
+            rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
+            __syncwarp();
+            if (!last_warp(slot)) {
+                if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
+                continue;
+            }
+            // the last warp: both K halves of every slab, in a fixed order
+#pragma unroll
+            for (int pp = 0; pp < kDownSlabs / 2; pp++) {
+                const float4 *r0 = reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp) * 32 + lane) * 8);
+                const float4 *r1 =
+                    reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp + 1) * 32 + lane) * 8);
+#pragma unroll
+                for (int sl = 0; sl < 2; sl++) {
+                    const float4 v0 = r0[sl], v1 = r1[sl];
+                    const float yv[4] = {v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w};
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const int tok = 2 * cq + (i & 1);
+                        const int row = (part * kDownSlabs + 2 * pp + sl) * kSlabRows + g + 8 * (i >> 1);
+                        if (tok < n) p.Y[(size_t)(slot0 + tok) * H + row] = 0.5f * yv[i];
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&empty[slot]);  // weights and partials consumed
+                // all 128 rows are stored: post the block for the combine warp
+                __threadfence_block();
+                const int idx = atomicAdd(misc + kMiscCombN, 1);
+                long long t0 = clock64();
+                while (idx - vmisc[kMiscCombSeen] >= kPubQ) {
+                    if (*abort_flag || clock64() - t0 > p.budget) {
+                        atomicCAS(p.err, 0, kErrTimeout);
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+                vmisc[kMiscCombQ + idx % kPubQ] = u * ndn + part + 1;
+            }
+        }
+    }
+    return jpos;
+}
+template <int kBits, bool kStaged>
+__global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int UB = unit_bytes(kBits);
     constexpr bool kMagic = kBits == 2;
@@ -458,7 +668,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     const int ne = e1 - e0;
     const int wbytes = ne * H * 4;                                 // router slice
     const int nwc = (wbytes + p.item_bytes - 1) / p.item_bytes;    // ring positions it takes
-    const int nxs = staged ? nsh * nsl : 0;                        // extras over the grid
+    const int nxs = kFExtras && staged ? nsh * nsl : 0;            // extras over the grid
     const int nx = cta < nxs ? (nxs - 1 - cta) / G + 1 : 0;        // this CTA's extras
     const size_t gu_bytes = (size_t)p.nseg_h * UB, dn_bytes = (size_t)kDownSlabs * p.nseg_i * UB;
 
@@ -486,7 +696,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     // the routed item list, once dispatch has run (same in every role)
     auto item_counts = [&](int &Ng, int &N2, int &ug0) {
         const int n_units = vmisc[kMiscNUnits];
-        ug0 = staged ? nsh : 0;  // with extras, the shared units' slabs are done already
+        ug0 = kFExtras && staged ? nsh : 0;  // with extras, the shared units' slabs are done already
         Ng = (n_units - ug0) * nsl;
         N2 = n_units * ndn;
     };
@@ -745,16 +955,20 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
 #pragma unroll
                     for (int cc = 0; cc < 4; cc++) {
                         const int col = part * kSlabRows * kDownSlabs + cc * 32 + lane;
+                        // unconditional loads (picks past k re-read the last
+                        // one): all k + 1 rows are in flight at once
                         float vv[kFMaxK];
 #pragma unroll
                         for (int r = 0; r < kFMaxK; r++)
-                            vv[r] = r < k ? __ldcg(p.Y + (size_t)sslot[sord[tt * k + r]] * H + col)
-                                          : 0.0f;
+                            vv[r] = __ldcg(p.Y + (size_t)sslot[sord[tt * k + (r < k ? r : k - 1)]] * H + col);
                         float acc2 = __ldcg(p.Y + (size_t)(Tk + tt) * H + col);
+                        // picks past k add an exact zero (weight 0, a finite
+                        // row), so every load is used and none is sunk into a
+                        // branch
 #pragma unroll
                         for (int r = 0; r < kFMaxK; r++)
-                            if (r < k) acc2 = fmaf(sw[sord[tt * k + r]], vv[r], acc2);
-                        if (ex) acc2 *= pow2f(2 * ex);
+                            acc2 = fmaf(r < k ? sw[sord[tt * k + r]] : 0.0f, vv[r], acc2);
+                        if (ex) acc2 = acc2 * pow2f(ex) * pow2f(ex);
                         __nv_bfloat16 *o = p.out + (size_t)tt * H + col;
                         const __nv_bfloat16 yb = __float2bfloat16_rn(acc2);
                         *o = p.residual ? __float2bfloat16_rn(__fadd_rn(__bfloat162float(*o),
@@ -806,36 +1020,20 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
                                    (uint32_t)px[64] | ((uint32_t)px[96] << 16));
             }
             if (warp < T) {
-                float ss = 0.0f;
-                for (int i = lane; i < H; i += 32) {
-                    const float v = __bfloat162float(xb[(size_t)warp * H + i]);
-                    ss = fmaf(v, v, ss);
-                }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                if (lane == 0) sex[warp] = p.w2 > 0.0f ? prescale_exp(sqrtf(ss) * p.w2 * 1.001f) : 0;
+                const int ex = token_prescale_warp(xb + (size_t)warp * H, H, p.w2, lane);
+                if (lane == 0) sex[warp] = ex;
             }
             compute_sync();
         }
     } else {
         // this CTA writes the expert operand of tokens cta, cta + G, ... for every CTA
         for (int t = cta; t < T; t += G) {
-            float ss = 0.0f;
-            for (int i = tid; i < H; i += kFCompute) {
-                const float v = __bfloat162float(p.x[(size_t)t * H + i]);
-                ss = fmaf(v, v, ss);
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            float *rs = red;
-            if (lane == 0) rs[warp] = ss;
-            compute_sync();
-            if (tid == 0) {
-                float s = 0.0f;
-                for (int w = 0; w < kFWarps; w++) s += rs[w];
-                const int ex = p.w2 > 0.0f ? prescale_exp(sqrtf(s) * p.w2 * 1.001f) : 0;
-                misc[kMiscTmp] = ex;
-                p.xex[t] = ex;
+            if (warp == 0) {
+                const int ex = token_prescale_warp(p.x + (size_t)t * H, H, p.w2, lane);
+                if (lane == 0) {
+                    misc[kMiscTmp] = ex;
+                    p.xex[t] = ex;
+                }
             }
             compute_sync();
             const int ex = misc[kMiscTmp];
@@ -859,59 +1057,68 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
         compute_sync();
         alive = *cflag != 0;
     }
-    if (alive && ne > 0) {
+    if (alive && ne > 0 && staged) {
+        // staged rows: one (token, expert) task per warp; lane l runs through
+        // its columns 128 s4 + 32 j + l in order (s4, then j), the loads of
+        // four steps in flight together
         const float4 *Ws = reinterpret_cast<const float4 *>(ring);  // [ne][H/128][32]
-        // staged rows: one (token, expert) task per warp; global rows: one
-        // token per warp, every expert of the CTA (each row read once)
-        const int per = staged ? 1 : ne;
-        const int ntask = staged ? T * ne : T;
-        for (int task = warp; task < ntask; task += kFWarps) {
-            const int t = staged ? task / ne : task;
-            const int eb = staged ? task % ne : 0;
-            for (int ee = eb; ee < eb + per; ee += 4) {
+        for (int task = warp; task < T * ne; task += kFWarps) {
+            const int t = task / ne, eb = task % ne;
+            const float4 *wr = Ws + (size_t)eb * ns4 * 32 + lane;
+            const uint2 *xr = xi + (size_t)t * ns4 * 32 + lane;
+            float acc = 0.0f;
+#pragma unroll 4
+            for (int s4 = 0; s4 < ns4; s4++) {
+                const uint2 v = xr[(size_t)s4 * 32];
+                const float4 w = wr[(size_t)s4 * 32];
+                acc = fmaf(__uint_as_float(v.x << 16), w.x, acc);
+                acc = fmaf(__uint_as_float(v.x & 0xffff0000u), w.y, acc);
+                acc = fmaf(__uint_as_float(v.y << 16), w.z, acc);
+                acc = fmaf(__uint_as_float(v.y & 0xffff0000u), w.w, acc);
+            }
+#pragma unroll
+            for (int sh = 16; sh >= 1; sh >>= 1)
+                acc = __fadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, sh));
+            if (lane == 0) {
+                const int e = e0 + eb;
+                p.logits[(size_t)t * E + e] = p.bias ? __fadd_rn(acc, p.bias[e]) : acc;
+            }
+        }
+    } else if (alive && ne > 0) {
+        // global rows: one token per warp, four of the CTA's experts at a time
+        // (each row read ne / 4 times, from L1); every load unconditional
+        // (a missing fourth expert repeats one and is not stored)
+        const float4 *Ws = reinterpret_cast<const float4 *>(ring);  // [ne][H/128][32]
+        for (int t = warp; t < T; t += kFWarps) {
+            const __nv_bfloat16 *xrow = p.x + (size_t)t * H + lane;
+            for (int ee = 0; ee < ne; ee += 4) {
+                const int nb = ne - ee < 4 ? ne - ee : 4;
+                const float4 *w0 = Ws + (size_t)ee * ns4 * 32 + lane;
+                const size_t st[4] = {0, (size_t)(1 < nb ? 1 : 0) * ns4 * 32,
+                                      (size_t)(2 < nb ? 2 : 0) * ns4 * 32,
+                                      (size_t)(3 < nb ? 3 : 0) * ns4 * 32};
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int s0 = 0; s0 < ns4; s0 += 4) {
-                    float xv[4][4];
+#pragma unroll 2
+                for (int s4 = 0; s4 < ns4; s4++) {
+                    float xv[4];
 #pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        const int s4 = s0 + c;
-                        if (staged) {
-                            const uint2 v = s4 < ns4 ? xi[((size_t)t * ns4 + s4) * 32 + lane]
-                                                     : make_uint2(0u, 0u);
-                            xv[c][0] = __uint_as_float(v.x << 16);
-                            xv[c][1] = __uint_as_float(v.x & 0xffff0000u);
-                            xv[c][2] = __uint_as_float(v.y << 16);
-                            xv[c][3] = __uint_as_float(v.y & 0xffff0000u);
-                        } else {
+                    for (int j = 0; j < 4; j++) xv[j] = __bfloat162float(xrow[128 * s4 + 32 * j]);
 #pragma unroll
-                            for (int j = 0; j < 4; j++)
-                                xv[c][j] = s4 < ns4 ? __bfloat162float(p.x[(size_t)t * H + 128 * s4 +
-                                                                           32 * j + lane])
-                                                    : 0.0f;
-                        }
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        if (s0 + c >= ns4) break;
-#pragma unroll
-                        for (int b = 0; b < 4; b++) {
-                            if (ee + b >= eb + per) break;
-                            const float4 w = Ws[((size_t)(ee + b) * ns4 + s0 + c) * 32 + lane];
-                            acc[b] = fmaf(xv[c][0], w.x, acc[b]);
-                            acc[b] = fmaf(xv[c][1], w.y, acc[b]);
-                            acc[b] = fmaf(xv[c][2], w.z, acc[b]);
-                            acc[b] = fmaf(xv[c][3], w.w, acc[b]);
-                        }
+                    for (int b = 0; b < 4; b++) {
+                        const float4 w = w0[st[b] + (size_t)s4 * 32];
+                        acc[b] = fmaf(xv[0], w.x, acc[b]);
+                        acc[b] = fmaf(xv[1], w.y, acc[b]);
+                        acc[b] = fmaf(xv[2], w.z, acc[b]);
+                        acc[b] = fmaf(xv[3], w.w, acc[b]);
                     }
                 }
 #pragma unroll
                 for (int b = 0; b < 4; b++) {
-                    if (ee + b >= eb + per) break;
                     float v = acc[b];
 #pragma unroll
-                    for (int s = 16; s >= 1; s >>= 1)
-                        v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, s));
-                    if (lane == 0) {
+                    for (int sh = 16; sh >= 1; sh >>= 1)
+                        v = __fadd_rn(v, __shfl_down_sync(0xffffffffu, v, sh));
+                    if (lane == 0 && b < nb) {
                         const int e = e0 + ee + b;
                         p.logits[(size_t)t * E + e] = p.bias ? __fadd_rn(v, p.bias[e]) : v;
                     }
@@ -921,234 +1128,58 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(lgbar);  // this warp's logits (and token rows) are stored
-    // the expert operand of the staged tokens and (2-bit) its block corrections
-    if (alive && staged) {
-        for (int i = tid; i < T * (H / 2); i += kFCompute) {
-            const int t = i / (H / 2), c = 2 * (i % (H / 2));
-            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(xb + (size_t)t * H + c);
-            __half2 h;
-            h.x = token_operand<kBits>(__bfloat162float(v.x), sex[t], c);
-            h.y = token_operand<kBits>(__bfloat162float(v.y), sex[t], c + 1);
-            *reinterpret_cast<__half2 *>(xs + (size_t)t * (H + 8) + c) = h;
-        }
-        if (kMagic)
-            for (int task = tid; task < T * nbh; task += kFCompute) {
-                const int t = task / nbh, b = task % nbh;
-                scorr[t * nbh + b] = block_correction<kBits>(xb + (size_t)t * H + 32 * b, sex[t]);
-            }
-    }
-    compute_sync();
+    compute_sync();                     // every warp is done with the router slice
     if (tid == 0)
         for (int s = 0; s < nwc; s++) mbar_arrive_cnt(&empty[s], kGWarps);  // router slice consumed
 
-    // ---- ring items: group gi (warps 8 gi .. 8 gi + 7) takes positions
-    // nwc + gi, nwc + gi + 2, ...; each of its warps takes a share of the item
-    //   gate/up slab: warp q an eighth of K of both the gate and the up slab;
-    //   down block: warp q the slabs 2 (q >> 1), 2 (q >> 1) + 1, half of K;
-    // and the last of the 8 to finish an item completes it.
-    const int gi = warp / kGWarps, q = warp % kGWarps;
-    int jpos = nwc + gi;
-    auto slot_exp = [&](int sl) -> int {  // the prescale exponent of a slot's token
-        const int t = sl < Tk ? slist[sl] : sl - Tk;
-        return staged ? sex[t] : __ldcg(p.xex + t);
-    };
-    auto slot_tok = [&](int sl) -> int { return sl < Tk ? slist[sl] : sl - Tk; };
-    // count this warp in for the item in `slot`; true for the last of the group
-    auto last_warp = [&](int slot) -> bool {
-        int old = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            old = atomicAdd(misc + kMiscGCnt + slot, 1);
-            if (old == kGWarps - 1) {
-                misc[kMiscGCnt + slot] = 0;  // before the slot can be refilled
-                __threadfence_block();
-            }
-        }
-        const bool last = __shfl_sync(0xffffffffu, old, 0) == kGWarps - 1;
-        __syncwarp();
-        return last;
-    };
-    auto run_items = [&](int stop) -> bool {  // false: aborted or end marker seen
-        for (; jpos < stop; jpos += kGroups) {
-            const int slot = jpos % p.ring;
-            if (!warp_fwait(&full[slot], (jpos / p.ring) & 1, p, abort_flag, lane)) return false;
-            const int meta = vmisc[kMiscMeta + slot];
-            if (meta == kItemEnd) return false;
-            const int kind = item_kind(meta);
-            int u, part, slot0, n;
-            if (kind == kKindExtra) {
-                const int i = meta & 0xfffffff;
-                u = i / nsl;
-                part = i % nsl;
-                slot0 = Tk + u * kFTile;
-                n = T - u * kFTile < kFTile ? T - u * kFTile : kFTile;
-            } else {
-                const int ug0 = staged ? nsh : 0;
-                if (kind == kKindGU) {
-                    const int it = meta & 0xfffffff;
-                    u = ug0 + it / nsl;
-                    part = it % nsl;
-                } else {
-                    const int d = meta & 0xfffff;
-                    u = d / ndn;
-                    part = d % ndn;
-                }
-                const int4 un = units[u];
-                slot0 = un.y;
-                n = un.z;
-            }
-            const uint8_t *w = ring + (size_t)slot * p.item_bytes;
-            float *rd = red + (size_t)slot * (kRedSlot / 4);  // [warp of group][lane][8]
-            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-            if (kind != kKindDown) {
-                // ---------------------------------- gate/up slab, K eighth q
-                // pairs of blocks: every range starts at an even block
-                const int b0 = 2 * (q * (nbh / 2) / 8), b1 = 2 * ((q + 1) * (nbh / 2) / 8);
-                // the lane's two token columns (columns past n repeat token 0)
-                const int ta = slot_tok(slot0 + (2 * cq < n ? 2 * cq : 0));
-                const int tb = slot_tok(slot0 + (2 * cq + 1 < n ? 2 * cq + 1 : 0));
-                if constexpr (kStaged) {
-                    const int r = lane & 7;
-                    const __half *rowp = xs + (size_t)slot_tok(slot0 + (r < n ? r : 0)) * (H + 8);
-                    slab2_blocks<kBits, kSrcSmem, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
-                                                          scorr + ta * nbh, scorr + tb * nbh, lane);
-                } else {
-                    const __half *rowp = p.x16 + (size_t)slot_tok(slot0 + (g < n ? g : 0)) * H;
-                    slab2_blocks<kBits, kSrcLdg, kMagic>(a0, a1, w, w + gu_bytes, b0, b1, rowp,
-                                                         p.corr + (size_t)ta * nbh,
-                                                         p.corr + (size_t)tb * nbh, lane);
-                }
-                float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
-                rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
-                rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
-                __syncwarp();
-                if (!last_warp(slot)) {
-                    if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
-                    continue;
-                }
-                // the last warp: the K eighths in a fixed order, then SwiGLU
-                float gs[4] = {0.f, 0.f, 0.f, 0.f}, us[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int j = 0; j < kGWarps; j++) {
-                    const float4 *rj = reinterpret_cast<const float4 *>(rd + ((size_t)j * 32 + lane) * 8);
-                    const float4 vg = rj[0], vu = rj[1];
-                    gs[0] += vg.x; gs[1] += vg.y; gs[2] += vg.z; gs[3] += vg.w;
-                    us[0] += vu.x; us[1] += vu.y; us[2] += vu.z; us[3] += vu.w;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);  // weights and partials consumed
-                // undo the operand factor: 2^8 (magic-offset form) or 2 (exact integers)
-                const float back = kMagic ? 1.0f / 256.0f : 0.5f;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int tok = 2 * cq + (i & 1);
-                    const float gv = gs[i] * back, uv = us[i] * back;
-                    // silu of the true gate value; the product stays in the
-                    // token's prescaled units (times 2^-2ex)
-                    const int ex = tok < n ? slot_exp(slot0 + tok) : 0;
-                    const float gt = ex ? gv * pow2f(ex) : gv;
-                    const float av = gv / (1.0f + expf(-gt)) * uv;
-                    const int row = part * kSlabRows + g + 8 * (i >> 1);
-                    if (tok < n) p.a[(size_t)(slot0 + tok) * p.Ip + row] = __float2half_rn(av);
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    // post the slab's unit for the publish warp (CTA scope)
-                    __threadfence_block();
-                    const int idx = atomicAdd(misc + kMiscPubN, 1);
-                    long long t0 = clock64();
-                    while (idx - vmisc[kMiscPubSeen] >= kPubQ) {
-                        if (*abort_flag || clock64() - t0 > p.budget) {
-                            atomicCAS(p.err, 0, kErrTimeout);
-                            *abort_flag = 1;
-                            break;
-                        }
-                    }
-                    vmisc[kMiscPubQ + idx % kPubQ] = u + 1;
-                }
-            } else {
-                // ------------------ down block: slabs 2 (q >> 1) + {0, 1}, K half q & 1
-                const int kd = (meta >> 20) & 0xff, b = kd % p.na;
-                if (!warp_fwait(&abar[b], (kd / p.na) & 1, p, abort_flag, lane)) return false;
-                const __half *abuf = abuf0 + (size_t)b * kFTile * (p.Ip + 8);
-                const int ar = lane & 7, pr = q >> 1, h = q & 1;
-                const __half *rowp = abuf + (size_t)(ar < n ? ar : 0) * (p.Ip + 8);
-                const uint8_t *s0 = w + (size_t)(2 * pr) * p.nseg_i * UB;
-                slab2_blocks<kBits, kSrcSmem, false>(a0, a1, s0, s0 + (size_t)p.nseg_i * UB,
-                                                     2 * (h * (nbi / 2) / 2), 2 * ((h + 1) * (nbi / 2) / 2), rowp, nullptr,
-                                                     nullptr, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&aempty[b]);  // activation rows consumed
-                float4 *rq = reinterpret_cast<float4 *>(rd + ((size_t)q * 32 + lane) * 8);
-                rq[0] = make_float4(a0[0], a0[1], a0[2], a0[3]);
-                rq[1] = make_float4(a1[0], a1[1], a1[2], a1[3]);
-                __syncwarp();
-                if (!last_warp(slot)) {
-                    if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
-                    continue;
-                }
-                // the last warp: both K halves of every slab, in a fixed order
-#pragma unroll
-                for (int pp = 0; pp < kDownSlabs / 2; pp++) {
-                    const float4 *r0 = reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp) * 32 + lane) * 8);
-                    const float4 *r1 =
-                        reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp + 1) * 32 + lane) * 8);
-#pragma unroll
-                    for (int sl = 0; sl < 2; sl++) {
-                        const float4 v0 = r0[sl], v1 = r1[sl];
-                        const float yv[4] = {v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w};
-#pragma unroll
-                        for (int i = 0; i < 4; i++) {
-                            const int tok = 2 * cq + (i & 1);
-                            const int row = (part * kDownSlabs + 2 * pp + sl) * kSlabRows + g + 8 * (i >> 1);
-                            if (tok < n) p.Y[(size_t)(slot0 + tok) * H + row] = 0.5f * yv[i];
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&empty[slot]);  // weights and partials consumed
-                    // all 128 rows are stored: post the block for the combine warp
-                    __threadfence_block();
-                    const int idx = atomicAdd(misc + kMiscCombN, 1);
-                    long long t0 = clock64();
-                    while (idx - vmisc[kMiscCombSeen] >= kPubQ) {
-                        if (*abort_flag || clock64() - t0 > p.budget) {
-                            atomicCAS(p.err, 0, kErrTimeout);
-                            *abort_flag = 1;
-                            break;
-                        }
-                    }
-                    vmisc[kMiscCombQ + idx % kPubQ] = u * ndn + part + 1;
-                }
-            }
-        }
-        return true;
-    };
+    // ring items: group gi (warps 8 gi .. 8 gi + 7) takes positions nwc + gi,
+    // nwc + gi + 2, ... (fused_run_items)
+    int jpos = nwc + warp / kGWarps;
 
-    // ---- the shared expert's slabs (no routing needed) while the grid barrier runs
-    if (alive) alive = run_items(nwc + nx);
-    // one verdict for all compute warps before the next compute-wide barriers
-    // (a warp that gave up above must not skip a barrier the others wait at)
-    if (!alive) misc[kMiscDead] = 1;
-    compute_sync();
-    alive = misc[kMiscDead] == 0;
-
-    // ---- top-k (picks in descending logit order; a tie to the lower id)
-    if (tid == 0) *cflag = alive && fwait(rdy, 0, p, abort_flag) ? 1 : 0;
-    compute_sync();
-    alive = *cflag != 0;
+    // ---- top-k (picks in descending logit order; a tie to the lower id).
+    // Up to kTopkLocalT tokens every CTA picks for every token: warp t < T
+    // takes token t once the grid barrier is through, while the other warps
+    // build the staged tokens' expert operand and (2-bit) its block
+    // corrections, which nothing reads before the first item.
     if (T <= kTopkLocalT) {
-        if (alive && warp < T) {
-            int pe;
-            float pw;
-            warp_topk(p.logits + (size_t)warp * E, E, k, lane, pe, pw);
-            if (lane < k) {
-                sidx[warp * k + lane] = pe;
-                sw[warp * k + lane] = pw;
+        if (warp < T) {
+            int ok = alive ? 1 : 0;
+            if (lane == 0 && ok) ok = fwait(rdy, 0, p, abort_flag) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok) {
+                int pe;
+                float pw;
+                warp_topk(p.logits + (size_t)warp * E, E, k, lane, pe, pw);
+                if (lane < k) {
+                    sidx[warp * k + lane] = pe;
+                    sw[warp * k + lane] = pw;
+                }
+            } else if (lane == 0) {
+                misc[kMiscDead] = 1;
             }
+        } else if (alive && staged) {
+            const int t0 = tid - 32 * T, nt = kFCompute - 32 * T;
+            for (int i = t0; i < T * (H / 2); i += nt) {
+                const int t = i / (H / 2), c = 2 * (i % (H / 2));
+                const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(xb + (size_t)t * H + c);
+                __half2 h;
+                h.x = token_operand<kBits>(__bfloat162float(v.x), sex[t], c);
+                h.y = token_operand<kBits>(__bfloat162float(v.y), sex[t], c + 1);
+                *reinterpret_cast<__half2 *>(xs + (size_t)t * (H + 8) + c) = h;
+            }
+            if (kMagic)
+                for (int task = t0; task < T * nbh; task += nt) {
+                    const int t = task / nbh, b = task % nbh;
+                    scorr[t * nbh + b] = block_correction<kBits>(xb + (size_t)t * H + 32 * b, sex[t]);
+                }
         }
+        if (!alive && lane == 0) misc[kMiscDead] = 1;
+        compute_sync();
+        alive = misc[kMiscDead] == 0;
     } else {
+        if (tid == 0) *cflag = alive && fwait(rdy, 0, p, abort_flag) ? 1 : 0;
+        compute_sync();
+        alive = *cflag != 0;
         if (alive && warp == 0 && cta < T) {
             int pe;
             float pw;
@@ -1176,7 +1207,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
 
     // ---- dispatch, identical in every CTA
     if (alive) {
-        for (int i = tid; i < Tk; i += kFCompute) atomicOr(&mask[sidx[i]], 1ull << (i / k));
+        for (int i = tid; i < Tk; i += kFCompute)
+            if (idx_ok(p.err, sidx[i], E)) atomicOr(&mask[sidx[i]], 1ull << (i / k));
         compute_sync();
         // one scan of (count << 16 | units): both sums stay below 2^16 (T k <= 1024)
         const int ept = (E + kFCompute - 1) / kFCompute, eb = tid * ept;
@@ -1210,7 +1242,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
         for (int i = tid; i < Tk; i += kFCompute) {
             const int t = i / k, ej = sidx[i];
             const int pos = soff[ej] + __popcll(mask[ej] & ((1ull << t) - 1ull));
-            slist[pos] = t;
+            if (idx_ok(p.err, pos, Tk)) slist[pos] = t;
             sslot[i] = pos;
             int rank = 0;
             for (int jj = 0; jj < k; jj++) rank += sidx[t * k + jj] < ej;
@@ -1223,7 +1255,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const FusedP
     grid_launch_dependents();
 
     // ---- routed slabs and down blocks, then the end marker
-    if (alive) run_items(1 << 30);
+    if (alive) fused_run_items<kBits, kStaged>(p, jpos, 1 << 30);
     __syncwarp();
     if (lane == 0) {
         __threadfence_block();

@@ -69,7 +69,8 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
     const uint8_t *__restrict__ routed, const uint8_t *__restrict__ shared, size_t expert_bytes,
     size_t mat_bytes, const int4 *__restrict__ units, const int *__restrict__ n_units,
     const int32_t *__restrict__ list, int Tk, int T, int E, const __nv_bfloat16 *__restrict__ x,
-    int H, int Ip, int xrows, int nsh, __half *__restrict__ a_out, int *err, long long budget) {
+    const int *__restrict__ xex, int H, int Ip, int xrows, int nsh, int srows,
+    __half *__restrict__ a_out, int *err, long long budget) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ float red[4][32][8];
     constexpr int UB = unit_bytes(kBits);
@@ -83,7 +84,7 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
     // shared CTAs signal by exiting.
     int4 un;
     if (u < nsh) {
-        const int n0 = T - u * kTile;
+        const int n0 = srows - u * kTile;  // the first srows tokens take the shared expert
         un = make_int4(E, Tk + u * kTile, n0 < kTile ? n0 : kTile, 0);
     } else {
         grid_dependency_wait();
@@ -92,6 +93,17 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
         un = units[u];
     }
     const int e = un.x, slot0 = un.y, n = un.z;
+    // lane j < n: token row j of the unit and its prescale factor 2^-xex
+    // (the exponents come from a kernel that completed before routing began)
+    int my_t = 0, my_ex = 0;
+    {
+        const int ln = threadIdx.x & 31;
+        if (ln < n) {
+            const int sl = slot0 + ln;
+            my_t = sl < Tk ? list[sl] : sl - Tk;
+            my_ex = xex[my_t];
+        }
+    }
     const uint8_t *wg = e == E ? shared : routed + (size_t)e * expert_bytes;
     const uint8_t *wu = wg + mat_bytes;
     const int nseg = H / kSegCols;
@@ -126,27 +138,27 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
 #pragma unroll
             for (int b = 0; b < 8; b++) {
                 const int idx = base + b * 32 + lane;
+                const int j = idx / per_row, i = idx % per_row;
+                const int t = __shfl_sync(0xffffffffu, my_t, j & 31);
                 v[b] = make_uint4(0, 0, 0, 0);
-                if (idx < nchunk) {
-                    const int j = idx / per_row, i = idx % per_row;
-                    if (j < n) {
-                        const int slot = slot0 + j;
-                        const int t = slot < Tk ? list[slot] : slot - Tk;
-                        v[b] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H +
-                                                                     sa * kSegCols) + i);
-                    }
-                }
+                if (idx < nchunk && j < n)
+                    v[b] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * H +
+                                                                 sa * kSegCols) + i);
             }
 #pragma unroll
             for (int b = 0; b < 8; b++) {
                 const int idx = base + b * 32 + lane;
-                if (idx >= nchunk) break;
                 const int j = idx / per_row, i = idx % per_row;
+                const float sc = pow2f(-__shfl_sync(0xffffffffu, my_ex, j & 31));
+                if (idx >= nchunk) break;
                 const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&v[b]);
                 uint4 o;
                 __half2 *h = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-                for (int q = 0; q < 4; q++) h[q] = __float22half2_rn(__bfloat1622float2(bb[q]));
+                for (int q = 0; q < 4; q++) {
+                    const float2 f = __bfloat1622float2(bb[q]);
+                    h[q] = __floats2half2_rn(f.x * sc, f.y * sc);
+                }
                 reinterpret_cast<uint4 *>(xb + j * pitch)[i] = o;
             }
         }
@@ -174,8 +186,8 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
                        red[3][lane][4 + i];
             gs *= 0.5f;  // the integers are 2(q - c): one factor 2 out
             us *= 0.5f;
-            float a = gs / (1.0f + expf(-gs)) * us;
             int tok = 2 * c + (i & 1);
+            const float a = swiglu_ps(gs, us, __shfl_sync(0xffffffffu, my_ex, tok));
             int row = slab * kSlabRows + g + 8 * (i >> 1);
             if (tok < n) a_out[(size_t)(slot0 + tok) * Ip + row] = __float2half_rn(a);
         }
@@ -267,16 +279,18 @@ static size_t down_smem(const Geometry &g, int xrows) {
 
 void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
                         const int *n_units, int units_max, const int32_t *list, int Tk, int T,
-                        const void *x, void *a_out, int *err, long long budget, cudaStream_t s) {
+                        const void *x, const int *xex, void *a_out, int *err, long long budget,
+                        cudaStream_t s, int shared_rows) {
     const int xrows = staged_rows(T);
-    const int nsh = (T + kTile - 1) / kTile;
+    const int nsh = ((shared_rows < 0 ? T : shared_rows) + kTile - 1) / kTile;
     size_t smem = gateup_smem(g, xrows);
     dim3 grid((unsigned)((size_t)units_max * (g.Ip / kSlabRows)));
     auto xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     auto ao = reinterpret_cast<__half *>(a_out);
     auto kern = g.bits == 2 ? gemv_gateup_kernel<2> : gemv_gateup_kernel<3>;
     launch_pdl(kern, grid, dim3(128), smem, s, w.routed, w.shared, g.expert_bytes, g.mat_bytes,
-               units, n_units, list, Tk, T, g.E, xb, g.H, g.Ip, xrows, nsh, ao, err, budget);
+               units, n_units, list, Tk, T, g.E, xb, xex, g.H, g.Ip, xrows, nsh,
+               shared_rows < 0 ? T : shared_rows, ao, err, budget);
 }
 
 void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *units,

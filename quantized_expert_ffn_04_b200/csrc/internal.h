@@ -22,6 +22,20 @@ struct Geometry {
 // -> GPU layout with Rp rows, Kp columns (zero weights in the padding).
 void launch_repack_matrix(const uint8_t *codes, const uint16_t *scales, int bits, int R, int K,
                           int Rp, int Kp, uint8_t *out, cudaStream_t s);
+// ---- ep.cu
+// Owner rank of expert e: floor(e n_ranks / E) (contiguous ranges).
+int ep_owner(int e, int E, int n_ranks);
+// dst row i = src row rows[i] (row_bytes a multiple of 16; rows outside
+// [0, n_src) are reported through err and skipped; with `keep`, rows i whose
+// keep[i] < 0 are skipped).
+void launch_gather_rows_bytes(const void *src, const int32_t *rows, int n, int n_src,
+                              int row_bytes, void *dst, int *err, cudaStream_t s,
+                              const int32_t *keep = nullptr);
+
+// Largest row L2 norm of a canonical matrix [R][K] (dequantised), max-folded
+// into *out_bits as float bits (start from 0).
+void launch_row_norm_max(const uint8_t *codes, const uint16_t *scales, int bits, int R, int K,
+                         unsigned *out_bits, cudaStream_t s);
 // Debug: dequantise rows [row0, row0+nrows) of a GPU-layout matrix with Kp
 // columns.  kind 0: exact fp32, kind 1: fp16 tensor-core operand (as float).
 void launch_debug_dequant(const uint8_t *mat, int bits, int Kp, int row0, int nrows, int ncols,
@@ -49,13 +63,14 @@ void dispatch_scratch_carve(void *base, int T, int E, DispatchScratch *d);
 int max_units(int T, int k, int E, int tile);
 void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *off,
                      int32_t *list, int32_t *slot, const DispatchScratch &ds, int4 *units,
-                     int *n_units, int tile, cudaStream_t s);
+                     int *n_units, int tile, cudaStream_t s, int *err = nullptr,
+                     int shared_rows = -1);
 
 // Top-k + dispatch for T <= kSmallMaxT tokens in a single CTA.
 constexpr int kSmallMaxT = 256;
 void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, float *w,
                         int32_t *cnt, int32_t *off, int32_t *list, int32_t *slot, int4 *units,
-                        int *n_units, int tile, cudaStream_t s);
+                        int *n_units, int tile, cudaStream_t s, int *err = nullptr);
 
 // Large batches: screened top-k from the split-weight screening GEMM D
 // ([T][R], hi part in columns [0, E), lo part in [E, 2E)) and exact recompute
@@ -71,24 +86,32 @@ struct ExpertWeights {
 };
 void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
                         const int *n_units, int units_max, const int32_t *list, int Tk, int T,
-                        const void *x, void *a_out, int *err, long long budget, cudaStream_t s);
+                        const void *x, const int *xex, void *a_out, int *err, long long budget,
+                        cudaStream_t s, int shared_rows = -1);
 void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
                       const int *n_units, int units_max, int T, const void *a, float *Y, int *err,
                       long long budget, cudaStream_t s);
 
 // ---- umma.cu (prefill)
-// x (bf16) -> x16 (fp16 copy), then gate/up (a: fp16 [slots][Ip]) and down
-// (Y: fp16 [slots][H]) on the tensor cores.  Units of up to 256 tokens.
+// x (bf16) -> x16 (fp16 prescaled copy, launch_prescale), then gate/up (a:
+// fp16 [slots][Ip], prescaled units) and down (Y: fp16 [slots][H], prescaled
+// units) on the tensor cores.  Units of up to 256 tokens.
 // The token operand xs is fp16 [slots][H] with slots = Tk + T: the routed
 // rows in slot order (launch_gather_rows), then the fp16 copy of x; a holds
 // `slots` rows too.  Each returns the launch status (an error also when the
 // tensor maps cannot be encoded).
 constexpr int kUmmaTile = 256;
+// Token prescale exponents xex[T] (common.cuh) and, when x16 is not NULL, the
+// prescaled fp16 operand x16[T][H] = fp16(x 2^-xex).
+void launch_prescale(const void *x, int T, int H, float w2, int *xex, void *x16, cudaStream_t s);
+// T: token rows in x16 (the checked build tests every list entry against it);
+// slot_ex[Tk + T] receives every slot's token exponent from xex.
 void launch_gather_rows(const int32_t *list, int Tk, const void *x16, void *xs, int H,
-                        cudaStream_t s);
+                        cudaStream_t s, int T, int *err, const int *xex, int *slot_ex);
 cudaError_t launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
                                const int *n_units, int units_max, int slots, const void *xs,
-                               void *a, int *err, long long budget, cudaStream_t s);
+                               const int *slot_ex, void *a, int *err, long long budget,
+                               cudaStream_t s);
 cudaError_t launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
                              const int *n_units, int units_max, int slots, const void *a, void *Y,
                              int *err, long long budget, cudaStream_t s);
@@ -133,9 +156,11 @@ cudaError_t fused_init_attributes(int max_smem);
 // out[t] = Y[Tk + t] + sum_j (ascending expert id) w[t][j] * Y[slot[t][j]]; bf16.
 // y_half: Y stored as fp16 (prefill) instead of fp32 (decode).  residual: h
 // (bf16, in place) <- bf16(f32(h) + f32(bf16(out))) instead of writing out.
+// xex: token prescale exponents (Y in prescaled units; the sum is taken
+// times 2^xex twice before the rounding), or NULL for unscaled Y.
 void launch_combine(const void *Y, bool y_half, const int32_t *idx, const float *w,
                     const int32_t *slot, int T, int k, int H, void *out, bool residual,
-                    cudaStream_t s);
+                    cudaStream_t s, int *err, const int *xex);
 void launch_rmsnorm(const void *h, void *xn, int T, int H, cudaStream_t s);
 
 // ---- selftest

@@ -74,6 +74,34 @@ void launch_repack_matrix(const uint8_t *codes, const uint16_t *scales, int bits
     repack_kernel<<<(unsigned)grid, bs, 0, s>>>(codes, scales, bits, R, K, Rp, Kp, out);
 }
 
+// ---- row norms for the token prescale: the largest L2 norm over the rows of
+// a canonical matrix [R][K] of dequantised weights d (q - c), folded into
+// *out_bits with an integer max (a non-negative float's bits order like the
+// float).  One warp per row.  The prescale only needs a bound, and it pads
+// this one by 0.1 %, far more than the rounding of the fp32 sum.
+__global__ void row_norm_max_kernel(const uint8_t *__restrict__ codes,
+                                    const uint16_t *__restrict__ scales, int bits, int R, int K,
+                                    unsigned *__restrict__ out_bits) {
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= R) return;
+    const float c = bits == 2 ? 1.5f : 3.5f;
+    float ss = 0.0f;
+    for (int col = lane; col < K; col += 32) {
+        const float d = __half2float(__ushort_as_half(scales[(size_t)row * (K / 32) + col / 32]));
+        const float w = d * ((float)canon_code(codes, bits, K, row, col) - c);
+        ss = fmaf(w, w, ss);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) atomicMax(out_bits, __float_as_uint(sqrtf(ss)));
+}
+
+void launch_row_norm_max(const uint8_t *codes, const uint16_t *scales, int bits, int R, int K,
+                         unsigned *out_bits, cudaStream_t s) {
+    row_norm_max_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(codes, scales, bits, R, K,
+                                                                 out_bits);
+}
+
 // ---- debug dequant: decode single weights from the GPU layout with the same
 // device routines the kernels use.
 template <int kBits>

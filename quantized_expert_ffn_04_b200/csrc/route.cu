@@ -338,7 +338,7 @@ __global__ __launch_bounds__(1024) void dispatch_scan_kernel(int T, int k, int E
                                                              int32_t *__restrict__ off,
                                                              int4 *__restrict__ units,
                                                              int *__restrict__ n_units,
-                                                             int tile) {
+                                                             int tile, int shared_rows) {
     const int e = threadIdx.x;  // E <= 1024
     int ce = 0;
     if (e < E)
@@ -362,14 +362,16 @@ __global__ __launch_bounds__(1024) void dispatch_scan_kernel(int T, int k, int E
     int us = block_exclusive_scan(nu, &utot);
     // shared-expert units first (their position is known before routing), then
     // the routed experts' units in ascending expert id
-    int nsh = (T + tile - 1) / tile;
+    // (the first shared_rows tokens get the shared expert; every token in a
+    // forward, fewer when rows are run for other ranks' tokens)
+    int nsh = (shared_rows + tile - 1) / tile;
     if (e < E)
         for (int i = 0; i < nu; i++) {
             int n = ce - i * tile;
             units[nsh + us + i] = make_int4(e, oe + i * tile, n < tile ? n : tile, 0);
         }
     for (int i = threadIdx.x; i < nsh; i += blockDim.x) {
-        int n = T - i * tile;
+        int n = shared_rows - i * tile;
         units[i] = make_int4(E, T * k + i * tile, n < tile ? n : tile, 0);
     }
     if (threadIdx.x == 0) *n_units = utot + nsh;
@@ -379,7 +381,7 @@ __global__ __launch_bounds__(1024) void dispatch_scan_kernel(int T, int k, int E
 __global__ __launch_bounds__(256) void dispatch_scatter_kernel(
     const int32_t *__restrict__ idx, int T, int k, int E, const int32_t *__restrict__ base,
     const uint32_t *__restrict__ bm, const int16_t *__restrict__ pre, int32_t *__restrict__ list,
-    int32_t *__restrict__ slot) {
+    int32_t *__restrict__ slot, int *err) {
     const int c = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = c * kChunk + threadIdx.x;
@@ -390,6 +392,7 @@ __global__ __launch_bounds__(256) void dispatch_scatter_kernel(
         if ((unsigned)e >= (unsigned)E) continue;
         size_t wi = ((size_t)c * 8 + warp) * E + e;
         int pos = base[(size_t)c * E + e] + pre[wi] + __popc(bm[wi] & below);
+        if (!idx_ok(err, pos, (long long)T * k)) continue;
         list[pos] = t;
         slot[(size_t)t * k + j] = pos;
     }
@@ -397,13 +400,15 @@ __global__ __launch_bounds__(256) void dispatch_scatter_kernel(
 
 void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *off,
                      int32_t *list, int32_t *slot, const DispatchScratch &ds, int4 *units,
-                     int *n_units, int tile, cudaStream_t s) {
+                     int *n_units, int tile, cudaStream_t s, int *err, int shared_rows) {
     int nc = n_chunks(T);
+    if (shared_rows < 0) shared_rows = T;
     size_t smem = (size_t)8 * E * 4;
     dispatch_count_kernel<<<nc, 256, smem, s>>>(idx, T, k, E, ds.hist, ds.bm, ds.pre);
     dispatch_scan_kernel<<<1, 1024, 0, s>>>(T, k, E, nc, ds.hist, cnt, off, units, n_units,
-                                            tile);
-    dispatch_scatter_kernel<<<nc, 256, 0, s>>>(idx, T, k, E, ds.hist, ds.bm, ds.pre, list, slot);
+                                            tile, shared_rows);
+    dispatch_scatter_kernel<<<nc, 256, 0, s>>>(idx, T, k, E, ds.hist, ds.bm, ds.pre, list, slot,
+                                               err);
 }
 
 // ============================================================== screened top-k
@@ -604,7 +609,7 @@ __global__ __launch_bounds__(1024) void route_small_kernel(
     const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx,
     float *__restrict__ wout, int32_t *__restrict__ cnt, int32_t *__restrict__ off,
     int32_t *__restrict__ list, int32_t *__restrict__ slot, int4 *__restrict__ units,
-    int *__restrict__ n_units, int tile) {
+    int *__restrict__ n_units, int tile, int *err) {
     extern __shared__ uint32_t sm[];
     grid_launch_dependents();  // the shared expert's gate/up CTAs may start now
     grid_dependency_wait();
@@ -660,7 +665,9 @@ __global__ __launch_bounds__(1024) void route_small_kernel(
         const uint32_t below = (1u << (t & 31)) - 1u;
         for (int j = 0; j < k; j++) {
             const int ej = sidx[t * k + j];
+            if (!idx_ok(err, ej, E)) continue;
             const int pos = soff[ej] + pre[g * E + ej] + __popc(bm[g * E + ej] & below);
+            if (!idx_ok(err, pos, (long long)T * k)) continue;
             list[pos] = t;
             slot[(size_t)t * k + j] = pos;
         }
@@ -669,10 +676,10 @@ __global__ __launch_bounds__(1024) void route_small_kernel(
 
 void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, float *w,
                         int32_t *cnt, int32_t *off, int32_t *list, int32_t *slot, int4 *units,
-                        int *n_units, int tile, cudaStream_t s) {
+                        int *n_units, int tile, cudaStream_t s, int *err) {
     size_t smem = ((size_t)8 * E * 2 + E + (size_t)T * k) * 4;
     launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, s, logits, T, E, k, idx, w, cnt,
-               off, list, slot, units, n_units, tile);
+               off, list, slot, units, n_units, tile, err);
 }
 
 cudaError_t route_init_attributes(int max_smem) {

@@ -60,11 +60,15 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[16], uint32_t &b
 static __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
                                         int &pick_e, float &pick_w) {
     uint32_t key[16];
-    const int nq = (E + 31) >> 5;
+    // every load is unconditional (entries past E re-read the last one) and
+    // its value is used unconditionally (masked, not branched on), so the
+    // compiler cannot sink the loads into branches: the 16 are in flight
+    // together instead of one after another
 #pragma unroll
     for (int q = 0; q < 16; q++) {
         const int e = q * 32 + lane;
-        key[q] = (q < nq && e < E) ? logit_key(__ldcg(row + e)) : 0u;
+        const float v = __ldcg(row + (e < E ? e : E - 1));
+        key[q] = logit_key(v) & (0u - (uint32_t)(e < E));
     }
     uint32_t bk;
     int bq;

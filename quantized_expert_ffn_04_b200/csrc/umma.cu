@@ -84,6 +84,7 @@ struct UmmaParams {
     int Tk;
     int K, nseg, n_rt;
     __half *out;        // gate/up: a [slots][Ip]; down: Y [slots][H]
+    const int *slot_ex; // gate/up: token prescale exponent of every slot
     float *out32;       // plain: D [T][n_rt * 128]
     int direct_T;       // plain: tiles are tokens [256u, 256u + 256) of T tokens
     int out_ld;
@@ -123,10 +124,12 @@ __device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, long l
 __device__ __forceinline__ uint32_t h2u(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
 __device__ __forceinline__ __half2 u2h(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
 
-// silu(g) * u with the fast exponential and division (the output is rounded
-// to fp16, far coarser than their error).
-__device__ __forceinline__ float swiglu(float g, float u) {
-    return __fdividef(g, 1.0f + __expf(-g)) * u;
+// silu(g) * u of a prescaled token (g, u times 2^-ex; the sigmoid takes the
+// true gate, the product stays times 2^-2ex) with the fast exponential and
+// division (the output is rounded to fp16, far coarser than their error).
+__device__ __forceinline__ float swiglu(float g, float u, int ex) {
+    const float gt = ex ? g * pow2f(ex) : g;
+    return __fdividef(g, 1.0f + __expf(-gt)) * u;
 }
 
 template <int kBits, int kMode>
@@ -406,16 +409,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                 if (kGateUp) {
                     float uv[32];
                     tmem_ld32(tb + kTN + nc * 32, uv);
+                    // lane j holds the prescale exponent of column j of the chunk
+                    const int exl = lane < cnt ? __ldg(p.slot_ex + slot0 + nc * 32 + lane) : 0;
                     if (cnt >= 32) {
 #pragma unroll
                         for (int j = 0; j < 32; j++)
-                            p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(swiglu(gv[j], uv[j]));
+                            p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(
+                                swiglu(gv[j], uv[j], __shfl_sync(0xffffffffu, exl, j)));
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; j++)
+                        for (int j = 0; j < 32; j++) {
+                            const int ex = __shfl_sync(0xffffffffu, exl, j);
                             if (j < cnt)
                                 p.out[o0 + (size_t)j * p.out_ld] =
-                                    __float2half_rn(swiglu(gv[j], uv[j]));
+                                    __float2half_rn(swiglu(gv[j], uv[j], ex));
+                        }
                     }
                 } else if (kMode == kModeDown) {
                     if (cnt >= 32) {
@@ -456,6 +464,40 @@ __global__ void to_half_kernel(const __nv_bfloat16 *__restrict__ x, __half *__re
 #pragma unroll
     for (int j = 0; j < 4; j++) h[j] = __float22half2_rn(__bfloat1622float2(b[j]));
     reinterpret_cast<uint4 *>(y)[i] = o;
+}
+
+// Token prescale (see common.cuh): one warp per token computes the exponent e
+// in the shared fixed order, stores it in xex[t] and, when x16 is given,
+// writes the expert operand fp16(x 2^-e) of the row.
+__global__ void prescale_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, float w2,
+                                int *__restrict__ xex, __half *__restrict__ x16) {
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const __nv_bfloat16 *row = x + (size_t)t * H;
+    const int e = token_prescale_warp(row, H, w2, lane);
+    if (lane == 0) xex[t] = e;
+    if (!x16) return;
+    const float sc = pow2f(-e);
+    const uint4 *src = reinterpret_cast<const uint4 *>(row);
+    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * H);
+    for (int i = lane; i < H / 8; i += 32) {
+        const uint4 v = src[i];
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
+        uint4 o;
+        __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float2 f = __bfloat1622float2(b[j]);
+            h[j] = __floats2half2_rn(f.x * sc, f.y * sc);
+        }
+        dst[i] = o;
+    }
+}
+
+void launch_prescale(const void *x, int T, int H, float w2, int *xex, void *x16, cudaStream_t s) {
+    if (T <= 0) return;
+    prescale_kernel<<<(unsigned)((T + 7) / 8), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(x), T, H, w2, xex, reinterpret_cast<__half *>(x16));
 }
 
 // ------------------------------------------------------------------- host
@@ -511,19 +553,28 @@ static cudaError_t run_umma(const UmmaParams &p, int max_tiles, cudaStream_t s) 
 // 16-byte copies); the shared expert's rows follow as x16 itself.
 __global__ void gather_rows_kernel(const int32_t *__restrict__ list, int Tk,
                                    const uint4 *__restrict__ x16, uint4 *__restrict__ xs,
-                                   int row16) {
+                                   int row16, int T, int *err, const int *__restrict__ xex,
+                                   int *__restrict__ slot_ex) {
     const int slot = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (slot >= Tk) return;
-    const uint4 *src = x16 + (size_t)__ldg(list + slot) * row16;
+    if (slot >= Tk + T) return;
+    if (slot >= Tk) {  // the shared expert's slots: rows already in place after the routed ones
+        if (lane == 0) slot_ex[slot] = xex[slot - Tk];
+        return;
+    }
+    const int t = __ldg(list + slot);
+    if (!idx_ok(err, t, T)) return;
+    if (lane == 0) slot_ex[slot] = xex[t];
+    const uint4 *src = x16 + (size_t)t * row16;
     uint4 *dst = xs + (size_t)slot * row16;
     for (int i = lane; i < row16; i += 32) dst[i] = __ldg(src + i);
 }
 
 void launch_gather_rows(const int32_t *list, int Tk, const void *x16, void *xs, int H,
-                        cudaStream_t s) {
-    if (Tk <= 0) return;
-    gather_rows_kernel<<<(unsigned)((Tk + 7) / 8), 256, 0, s>>>(
-        list, Tk, reinterpret_cast<const uint4 *>(x16), reinterpret_cast<uint4 *>(xs), H / 8);
+                        cudaStream_t s, int T, int *err, const int *xex, int *slot_ex) {
+    if (Tk + T <= 0) return;
+    gather_rows_kernel<<<(unsigned)((Tk + T + 7) / 8), 256, 0, s>>>(
+        list, Tk, reinterpret_cast<const uint4 *>(x16), reinterpret_cast<uint4 *>(xs), H / 8,
+        T, err, xex, slot_ex);
 }
 
 void launch_to_half(const void *x, void *x16, size_t n, cudaStream_t s) {
@@ -552,9 +603,11 @@ static UmmaParams base_params(const Geometry &g, const ExpertWeights &w, const i
 
 cudaError_t launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const int4 *units,
                                const int *n_units, int units_max, int slots, const void *xs,
-                               void *a, int *err, long long budget, cudaStream_t s) {
+                               const int *slot_ex, void *a, int *err, long long budget,
+                               cudaStream_t s) {
     // A = Wg, Wu (Ip rows, K = H); B = token rows by slot
     UmmaParams p = base_params(g, w, units, n_units, nullptr, 0, err, budget);
+    p.slot_ex = slot_ex;
     cudaError_t e = encode_fp16_map(&p.tm_b, xs, g.H, slots, kBoxRows);
     if (e != cudaSuccess) return e;
     p.mat_off = 0;

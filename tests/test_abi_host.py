@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     text = open(os.path.join(ROOT, "include", "strata_moe.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(strata_moe_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(strata_(?:moe|ep)_\w+)\s*\(", text)))
 
 
 def test_header_symbols_exported():
@@ -27,6 +27,15 @@ def test_header_symbols_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert sorted(qe.SYMBOLS) == names
+
+
+def test_checked_build_exports_the_same_symbols():
+    """The checked variant (-DSTRATA_CHECKS=1) is the same ABI."""
+    path = os.path.join(os.path.dirname(qe.LIB_PATH), "libstrata_moe_checked.so")
+    assert os.path.exists(path), "build the checked variant (__graft_entry__.build())"
+    lib = C.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
 
 
 def test_version_and_last_error():
