@@ -79,6 +79,12 @@ FLASH3 = LayerShape(hidden=2560, n_experts=512, top_k=10, inter=640, bits=3, rou
 # how the experts are chosen is not on the path
 PRUNED256 = LayerShape(hidden=2560, n_experts=256, top_k=10, inter=640, bits=2,
                        router_bias=True)
+# 1-bit codes (w = d (q - 0.5)): the pages mention a 1-bit Coder quant
+# ("Open-Source Strata Runs a 125-Billion-Parameter Model ...", Key Facts
+# item 4) without a layout; read as the same block-32 family, here on the
+# pruned 256-expert Coder shape, and a tiny layer for the oracle's pins
+CODER1 = LayerShape(hidden=2560, n_experts=256, top_k=10, inter=640, bits=1, router_bias=True)
+TINY1 = LayerShape(hidden=256, n_experts=16, top_k=2, inter=64, bits=1, router_bias=False)
 STACK_LAYERS = 48
 
 

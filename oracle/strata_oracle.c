@@ -130,23 +130,27 @@ uint16_t orc_f64_to_f16(double v)
 /* ------------------------------------------------------------------------ */
 
 /* Code q of element j (0..31) of one block.
+ *  1-bit: 4 bytes; element j is bit j%8 of byte j/8.
  *  2-bit: 8 bytes; element j sits in bits 2*(j%4) .. 2*(j%4)+1 of byte j/4.
  *  3-bit: 12 bytes read as one little-endian 96-bit integer; element j sits in
- *         bits 3j .. 3j+2. */
+ *         bits 3j .. 3j+2.
+ * (All three: element j occupies bits bits*j .. bits*j+bits-1 of the block
+ * read as one little-endian integer.) */
 int orc_code(const uint8_t *block, int bits, int j)
 {
     if (bits == 2)
         return (block[j >> 2] >> (2 * (j & 3))) & 3;
-    int bit = 3 * j, q = 0;
-    for (int b = 0; b < 3; b++) {
+    int bit = bits * j, q = 0;
+    for (int b = 0; b < bits; b++) {
         int p = bit + b;
         q |= ((block[p >> 3] >> (p & 7)) & 1) << b;
     }
     return q;
 }
 
-/* Centre of the code range: w = d * (q - centre). */
-static double code_centre(int bits) { return bits == 2 ? 1.5 : 3.5; }
+/* Centre of the code range: w = d * (q - centre), centre = (2^bits - 1) / 2
+ * (0.5, 1.5, 3.5 for 1, 2, 3 bits). */
+static double code_centre(int bits) { return ((double)(1 << bits) - 1.0) / 2.0; }
 
 /* Exact dequantised weight (row r, column c) of a rows x cols matrix stored in
  * the packed format: codes [rows][cols/32][4*bits], scales [rows][cols/32]. */
@@ -386,7 +390,7 @@ int orc_moe_forward(int H, int E, int k, int I, int bits, const uint8_t *codes,
                     const uint16_t *x, int T, const int32_t *sel, int n_sel, uint16_t *y_bf16,
                     double *y_f64, int32_t *idx, double *w)
 {
-    if ((bits != 2 && bits != 3) || H % 32 || I % 32 || k < 1 || k > E)
+    if (bits < 1 || bits > 3 || H % 32 || I % 32 || k < 1 || k > E)
         return -1;
     orc_layer L = {H, E, k, I, bits, codes, scales, router_w, router_b, shared_codes,
                    shared_scales};

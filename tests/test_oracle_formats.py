@@ -70,7 +70,7 @@ def test_bf16_rounding_worked_and_brute_force():
     assert np.array_equal(got, npref.round_bf16_rne(v))
 
 
-@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("bits", [1, 2, 3])
 def test_code_extraction_matches_bit_serial_reader(bits):
     rng = np.random.default_rng(bits)
     rows, cols = 8, 128
@@ -83,7 +83,7 @@ def test_code_extraction_matches_bit_serial_reader(bits):
             assert got == list(ref[r, b * 32:(b + 1) * 32])
 
 
-@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("bits", [1, 2, 3])
 def test_dequant_matrix_matches_numpy_decoder(bits):
     shape = gen.LayerShape(hidden=256, n_experts=2, top_k=1, inter=64, bits=bits)
     w = gen.layer_weights(shape, seed=11)

@@ -45,7 +45,8 @@ def _logit_gaps(logits, k):
 
 
 @pytest.mark.parametrize("shape", [TINY, gen.LayerShape(hidden=128, n_experts=6, top_k=3,
-                                                        inter=32, bits=3, router_bias=True)])
+                                                        inter=32, bits=3, router_bias=True),
+                                   gen.TINY1])
 def test_brute_force_dense_masked(shape):
     layer = gen.layer_weights(shape, seed=0)
     x = gen.hidden(8, shape.hidden, seed=0)
