@@ -48,6 +48,10 @@ WORKLOADS = {
     "tiny-t8": (gen.TINY, 8, "tiny MoE layer H256 E16 k2 I64, T=8"),
     "pruned256-t4": (gen.PRUNED256, 4, "pruned 256-expert build of the Flash-Next-shaped layer, "
                                        "decode T=4, 2-bit block-32"),
+    "coder1-t4": (gen.CODER1, 4, "pruned 256-expert Coder build of the Flash-Next-shaped layer, "
+                                 "decode T=4, 1-bit block-32"),
+    "coder1-t8192": (gen.CODER1, 8192, "pruned 256-expert Coder build of the Flash-Next-shaped "
+                                       "layer, prefill chunk T=8192, 1-bit block-32"),
     # 48-layer expert stack: h <- h + MoE(RMSNorm(h)) through 48 resident layers
     "stack48-t4": (gen.FLASH2, 4, "48-layer Flash-Next-shaped expert stack (~37 GB of 2-bit "
                                   "experts resident), decode T=4"),

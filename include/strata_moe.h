@@ -57,7 +57,7 @@ typedef struct strata_moe *strata_moe_t; /* opaque, library-owned */
 
 /* Layer shape.  Supported: hidden % 128 == 0 and 128 <= hidden <= 6144;
  * 1 <= n_experts <= 1024; 1 <= top_k <= min(n_experts, 32); inter % 32 == 0
- * and 32 <= inter <= 4096; quant_bits in {2, 3}; block == 32;
+ * and 32 <= inter <= 4096; quant_bits in {1, 2, 3}; block == 32;
  * 1 <= max_tokens <= 65536.  Anything else returns STRATA_ERR_UNSUPPORTED
  * (or INVALID_ARG for non-positive values). */
 typedef struct {
@@ -65,7 +65,8 @@ typedef struct {
     int32_t n_experts;       /* E */
     int32_t top_k;           /* k routed experts per token */
     int32_t inter;           /* I, SwiGLU intermediate size */
-    int32_t quant_bits;      /* 2: w = d*(q-1.5), q in 0..3;  3: w = d*(q-3.5), q in 0..7 */
+    int32_t quant_bits;      /* 1: w = d*(q-0.5), q in 0..1;  2: w = d*(q-1.5), q in 0..3;
+                                3: w = d*(q-3.5), q in 0..7 */
     int32_t block;           /* quantisation block along the input dimension: 32 */
     int32_t max_tokens;      /* largest T accepted; sizes the handle's workspace */
     int32_t has_router_bias; /* 1: router_b is read; 0: logits carry no bias */
@@ -76,6 +77,9 @@ typedef struct {
  * Each expert has three matrices, in this order: 0 gate [I][H], 1 up [I][H],
  * 2 down [H][I], all row-major [out][in] and quantised along `in` in blocks of
  * 32 elements.  A block is 4*bits bytes of codes plus one fp16 scale d:
+ *   1-bit: element j is bit j%8 of byte j/8 (the pages mention a 1-bit quant,
+ *          "Open-Source Strata Runs a 125-Billion-Parameter Model ...", Key
+ *          Facts item 4, with no layout: read as the same block-32 family);
  *   2-bit: element j in bits 2*(j%4)..2*(j%4)+1 of byte j/4;
  *   3-bit: the 12 bytes form one little-endian 96-bit integer, element j in
  *          bits 3j..3j+2.
@@ -184,7 +188,8 @@ strata_status strata_moe_debug_dequant(strata_moe_t h, int expert, int mat, int 
  * expert id to the owner -> the owner runs strata_moe_expert_rows on what it
  * got -> outputs back in the same order -> strata_moe_combine_rows.  Each
  * expert output depends on one token row and one expert only, so the result
- * equals the one-GPU forward bit for bit (prefill = T > 64, as there). */
+ * equals the one-GPU forward on the same kernels bit for bit (prefill =
+ * T > 64; below, the decode GEMV chain, STRATA_OPT_PATH 1). */
 strata_status strata_ep_expert_range(int rank, int n_ranks, int n_experts, int32_t *e_begin,
                                      int32_t *e_end);
 
@@ -229,6 +234,17 @@ strata_status strata_moe_combine_rows(strata_moe_t h, const void *x_dev, int T,
                                       const int32_t *idx_dev, const float *w_dev,
                                       const int32_t *slot_dev, const void *y_dev, int prefill,
                                       void *out_dev, void *stream);
+
+/* Test hook of the large-batch router (T > 256): the approximate logits
+ * a[t][e] of its tensor-core screening GEMM (fp16 split of W, fp32
+ * accumulation, plus the bias) and each token's error bound eps[t], so that a
+ * test can measure |a - l| against eps for the exact fixed-order logits l
+ * (the screen keeps every expert with a >= a_(k) - 2 eps; a token whose bound
+ * is not finite or that has an entry beyond 65504 gets eps = 0 and keeps every
+ * expert).  a_host float [T][E], eps_host float [T].  Needs a handle with
+ * max_tokens > 256.  Synchronous. */
+strata_status strata_moe_debug_screen(strata_moe_t h, const void *x_dev, int T, float *a_host,
+                                      float *eps_host);
 
 /* Test hooks for the out-of-memory paths.  Every device and pinned host
  * allocation of the library goes through one counter.

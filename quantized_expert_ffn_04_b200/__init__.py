@@ -36,7 +36,7 @@ SYMBOLS = ("strata_moe_create", "strata_moe_destroy", "strata_moe_route", "strat
            "strata_moe_set_probe", "strata_moe_launch_count", "strata_moe_route_noalloc",
            "strata_moe_debug_fail_alloc", "strata_moe_debug_live_allocs",
            "strata_ep_expert_range", "strata_ep_plan", "strata_ep_gather_rows",
-           "strata_moe_expert_rows", "strata_moe_combine_rows")
+           "strata_moe_expert_rows", "strata_moe_combine_rows", "strata_moe_debug_screen")
 
 
 class strata_moe_config(C.Structure):
@@ -74,6 +74,7 @@ _sig = {
     "strata_moe_launch_count": [_P, _I],
     "strata_moe_route_noalloc": [_P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P],
     "strata_moe_debug_fail_alloc": [_I64],
+    "strata_moe_debug_screen": [_P, _P, _I, _P, _P],
     "strata_ep_expert_range": [_I, _I, _I, _P, _P],
     "strata_ep_plan": [_P, _I, _I, _I, _I, _P, _P, _P],
     "strata_ep_gather_rows": [_P, _P, _I, _I, _I, _P, _P],
@@ -179,6 +180,10 @@ def strata_moe_expert_rows(h, x, ids, n, n_shared, prefill, y, yshared, stream=N
 
 def strata_moe_combine_rows(h, x, T, idx, w, slot, y, prefill, out, stream=None) -> None:
     _check(_lib.strata_moe_combine_rows(h, x, T, idx, w, slot, y, int(prefill), out, stream))
+
+
+def strata_moe_debug_screen(h, x, T, a_host, eps_host) -> None:
+    _check(_lib.strata_moe_debug_screen(h, x, T, a_host, eps_host))
 
 
 def strata_moe_debug_fail_alloc(n) -> None:

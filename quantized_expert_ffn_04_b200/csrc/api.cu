@@ -3,6 +3,7 @@
 // stream.  Every step of the layer runs in this library's kernels; there is no
 // host fallback.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <stdarg.h>
 #include <stdio.h>
@@ -169,8 +170,8 @@ strata_status validate_config(const strata_moe_config *c) {
         c->max_tokens <= 0 || c->block <= 0)
         return fail(STRATA_ERR_INVALID_ARG, "config fields must be positive");
     if (c->block != 32) return fail(STRATA_ERR_UNSUPPORTED, "block must be 32 (got %d)", c->block);
-    if (c->quant_bits != 2 && c->quant_bits != 3)
-        return fail(STRATA_ERR_UNSUPPORTED, "quant_bits must be 2 or 3 (got %d)", c->quant_bits);
+    if (c->quant_bits < 1 || c->quant_bits > 3)
+        return fail(STRATA_ERR_UNSUPPORTED, "quant_bits must be 1, 2 or 3 (got %d)", c->quant_bits);
     if (c->hidden % 128 || c->hidden > 6144)
         return fail(STRATA_ERR_UNSUPPORTED, "hidden must be a multiple of 128 and <= 6144 (got %d)",
                     c->hidden);
@@ -279,7 +280,16 @@ strata_status check_tokens(strata_moe_t h, int T) {
 
 enum { kStRouter, kStTopk, kStDispatch, kStGateUp, kStDown, kStCombine };
 
+// Stage names of the NVTX ranges (one range per stage's launches on the
+// host timeline; a profiler lines them up with the kernels).
+const char *const kStageName[] = {"strata router", "strata top-k + dispatch", "strata dispatch",
+                                  "strata gate/up", "strata down", "strata combine"};
+
 void probe(strata_moe_t h, int stage, bool begin, cudaStream_t s) {
+    if (begin)
+        nvtxRangePushA(kStageName[stage]);
+    else
+        nvtxRangePop();
     cudaEvent_t e = begin ? h->probe_begin[stage] : h->probe_end[stage];
     if (!e) return;
     // inside a stream capture the record must become an event node of the graph
@@ -837,6 +847,8 @@ strata_status strata_moe_expert_rows(strata_moe_t h, const void *x_dev, const in
     if (n == 0) return STRATA_OK;
     if (!x_dev || !ids_dev || !y_dev || (n_shared > 0 && !yshared_dev))
         return fail(STRATA_ERR_INVALID_ARG, "NULL buffer");
+    if ((((uintptr_t)x_dev) | ((uintptr_t)y_dev) | ((uintptr_t)yshared_dev)) & 15)
+        return fail(STRATA_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
     DeviceGuard guard(h->device);
     cudaStream_t s = (cudaStream_t)stream;
     const Geometry &g = h->geo;
@@ -884,6 +896,8 @@ strata_status strata_moe_combine_rows(strata_moe_t h, const void *x_dev, int T,
     if (T == 0) return STRATA_OK;
     if (!x_dev || !idx_dev || !w_dev || !slot_dev || !y_dev || !out_dev)
         return fail(STRATA_ERR_INVALID_ARG, "NULL buffer");
+    if ((((uintptr_t)x_dev) | ((uintptr_t)y_dev) | ((uintptr_t)out_dev)) & 15)
+        return fail(STRATA_ERR_INVALID_ARG, "x, y and out must be 16-byte aligned");
     DeviceGuard guard(h->device);
     cudaStream_t s = (cudaStream_t)stream;
     const Geometry &g = h->geo;
@@ -891,6 +905,39 @@ strata_status strata_moe_combine_rows(strata_moe_t h, const void *x_dev, int T,
     launch_combine(y_dev, prefill != 0, idx_dev, w_dev, slot_dev, T, g.k, g.H, out_dev, false, s,
                    h->err, h->xex);
     return check_launch("combine rows");
+}
+
+strata_status strata_moe_debug_screen(strata_moe_t h, const void *x_dev, int T, float *a_host,
+                                      float *eps_host) {
+    if (!h || !x_dev || !a_host || !eps_host) return fail(STRATA_ERR_INVALID_ARG, "NULL argument");
+    strata_status st = check_tokens(h, T);
+    if (st != STRATA_OK) return st;
+    if (h->cfg.max_tokens <= kSmallMaxT)
+        return fail(STRATA_ERR_UNSUPPORTED, "the screening router needs max_tokens > %d",
+                    kSmallMaxT);
+    if (T == 0) return STRATA_OK;
+    DeviceGuard guard(h->device);
+    const Geometry &g = h->geo;
+    float *a = nullptr, *eps = nullptr;
+    if (dev_malloc(&a, (size_t)T * g.E * 4) != cudaSuccess ||
+        dev_malloc(&eps, (size_t)T * 4) != cudaSuccess) {
+        dev_free(a);
+        return fail(STRATA_ERR_OOM, "debug screen buffers");
+    }
+    launch_to_half(x_dev, x16_of(h, T), (size_t)T * g.H, 0);
+    cudaError_t ce = launch_umma_plain(h->router_split, h->router_rows, x16_of(h, T), T, g.H,
+                                       h->dsplit, h->err, h->budget, 0);
+    if (ce == cudaSuccess) {
+        launch_screen_debug(h->dsplit, h->router_rows, x_dev, T, g.H, h->router_b, g.E,
+                            h->screen_gam, h->screen_wmax, h->screen_bmax, a, eps, 0);
+        ce = cudaGetLastError();
+    }
+    if (ce == cudaSuccess) ce = cudaMemcpy(a_host, a, (size_t)T * g.E * 4, cudaMemcpyDeviceToHost);
+    if (ce == cudaSuccess) ce = cudaMemcpy(eps_host, eps, (size_t)T * 4, cudaMemcpyDeviceToHost);
+    dev_free(a);
+    dev_free(eps);
+    if (ce != cudaSuccess) return cuda_fail(ce, "debug screen");
+    return strata_moe_sync_status(h, nullptr);
 }
 
 strata_status strata_moe_debug_fail_alloc(int64_t n) {

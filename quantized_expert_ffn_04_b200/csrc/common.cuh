@@ -34,6 +34,11 @@ namespace strata {
 //                     fragment: r=0 (g, 2c|2c+1), r=1 (g+8, 2c|2c+1),
 //                     r=2 (g, 2c+8|2c+9), r=3 (g+8, 2c+8|2c+9); col relative to
 //                     16*s inside the block.
+//   1-bit units keep the same positions with half the words: [0, 256), lane
+//                     L owns 8 bytes = 2 words, word h holds block 2h's codes
+//                     at the 2-bit positions P, 16 + P and block 2h+1's one
+//                     bit higher (P + 1, 17 + P), so block 2h+1 decodes from
+//                     the word shifted right by one.
 //     [512, 768)      3-bit only: high bit of every code, lane L owns 8 bytes =
 //                     2 words; word h holds blocks 2h (bits r', 16+r') and
 //                     2h+1 (bits 8+r', 24+r').
@@ -49,8 +54,22 @@ __host__ __device__ constexpr int code_pos(int bits, int rp) {
                      : 2 * rp;
 }
 
+// Code bytes of a unit below the 3-bit high bits and the scales.
+__host__ __device__ constexpr int lo_bytes(int bits) { return bits == 1 ? kLoBytes / 2 : kLoBytes; }
+// Offset of the scales inside a unit.
+__host__ __device__ constexpr int scale_off(int bits) {
+    return lo_bytes(bits) + (bits == 3 ? kHiBytes : 0);
+}
 __host__ __device__ constexpr int unit_bytes(int bits) {
-    return kLoBytes + (bits == 3 ? kHiBytes : 0) + kScaleBytes;
+    return scale_off(bits) + kScaleBytes;
+}
+// The code word of block b (0..3) of a unit for this lane, in the 2-bit
+// positions (1-bit: the shared word, shifted for the odd block).
+template <int kBits>
+__device__ __forceinline__ uint32_t unit_word(const uint8_t *unit, int lane, int b) {
+    if (kBits == 1)
+        return *reinterpret_cast<const uint32_t *>(unit + lane * 8 + (b >> 1) * 4) >> (b & 1);
+    return *reinterpret_cast<const uint32_t *>(unit + lane * 16 + b * 4);
 }
 
 // ---------------------------------------------------------------- errors
@@ -445,6 +464,16 @@ STRATA_DEV uint32_t dq2_mul(int j) {
 STRATA_DEV uint32_t dq2_off(int j) {
     return j == 0 ? 0xE006E006u : j == 1 ? 0xD818D818u : j == 2 ? 0xD060D060u : 0xC980C980u;
 }
+// 1-bit: -(2^(11 - P) + 1), so h 2^(1 - P) + off = 2q - 1 (P = 2 + 2j).
+STRATA_DEV uint32_t dq1_off(int j) {
+    return j == 0 ? 0xE002E002u : j == 1 ? 0xD808D808u : j == 2 ? 0xD020D020u : 0xC880C880u;
+}
+// The code mask of column group j at mantissa bit P = 2 + 2j: two bits
+// (2-bit) or one (1-bit), in both halves.
+template <int kBits>
+__host__ __device__ constexpr uint32_t dq_mask(int j) {
+    return (kBits == 2 ? 3u : 1u) * ((1u << (2 + 2 * j)) | (1u << (18 + 2 * j)));
+}
 
 // ---------------------------------------------------------- token prescale
 // The expert kernels take the token operand in fp16, whose range (largest
@@ -486,20 +515,40 @@ STRATA_DEV int prescale_final(int em, float ss, float w2) {
     const int e = em + d;
     return e > 120 ? 120 : e;
 }
-// The prescale exponent of one bf16 row of length H, computed by one warp in
-// one fixed order (lane l takes i = l, l + 32, ... with fma, then a halving
-// tree), so every kernel that needs it gets the same e.  All lanes return e.
+// The prescale exponent of one bf16 row of length H (a multiple of 8, the row
+// 16-byte aligned), computed by one warp in one fixed order: lane l takes the
+// 8-element groups l, l + 32, ... (16-byte loads, four in flight), each group
+// in ascending order with fma, then a halving tree.  Every kernel that needs
+// e calls this, so they all get the same e.  All lanes return e.
+STRATA_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+STRATA_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 STRATA_DEV int token_prescale_warp(const __nv_bfloat16 *row, int H, float w2, int lane) {
+    const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
+    const int n8 = H >> 3;
     float m = 0.0f;
-    for (int i = lane; i < H; i += 32) m = fmaxf(m, fabsf(__bfloat162float(row[i])));
+#pragma unroll 4
+    for (int i = lane; i < n8; i += 32) {
+        const uint4 v = r4[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const int em = prescale_emax(m);
     const float sc = pow2f(-em);
     float ss = 0.0f;
-    for (int i = lane; i < H; i += 32) {
-        const float v = __bfloat162float(row[i]) * sc;
-        ss = fmaf(v, v, ss);
+#pragma unroll 4
+    for (int i = lane; i < n8; i += 32) {
+        const uint4 v = r4[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float a = bf16_lo(w[j]) * sc, b = bf16_hi(w[j]) * sc;
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -518,18 +567,21 @@ STRATA_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
     return d;
 }
 
-// Register r' (0..7) of a 2-bit block word: fp16 pair of 2q - 3.
+// Register r' (0..7) of a 2-bit (1-bit) block word: fp16 pair of 2q - 3
+// (2q - 1).
+template <int kBits = 2>
 STRATA_DEV uint32_t dq2_pair(uint32_t w, int rp) {
     const uint32_t src = (rp & 1) ? (rp == 7 ? (w << 8) : (w >> 8)) : w;
     const int j = rp >> 1;  // the code sits at mantissa bit 2 j + 2
-    const uint32_t mask = (3u << (2 * j + 2)) | (3u << (16 + 2 * j + 2));
-    return hfma2_u32((src & mask) | 0x64006400u, dq2_mul(j), dq2_off(j));
+    return hfma2_u32((src & dq_mask<kBits>(j)) | 0x64006400u, dq2_mul(j),
+                     kBits == 2 ? dq2_off(j) : dq1_off(j));
 }
 
 // One 32-wide block of a 2-bit matrix against 8 token columns, fp16
 // operands, fp32 result d (fresh): the 8 fragment registers are extracted from
 // word w (2 shifts, 8 mask/or, 8 packed fma) and fed to two m16n8k16 mma in
 // one asm block so they land directly in the operand registers.
+template <int kBits = 2>
 STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, uint32_t b2,
                            uint32_t b3) {
     // pure register arithmetic (not volatile): the compiler may schedule the
@@ -541,14 +593,14 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
         "mov.f32 z, 0f00000000;\n\t"
         "shr.b32 s8, %4, 8;\n\t"
         "shl.b32 s2, %4, 8;\n\t"
-        "lop3.b32 h0, %4, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h1, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h2, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h3, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h4, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h5, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h6, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h7, s2, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h0, %4, %17, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h1, s8, %17, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h2, %4, %18, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h3, s8, %18, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h4, %4, %19, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h5, s8, %19, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h6, %4, %20, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h7, s2, %20, 0x64006400, 0xEA;\n\t"
         "fma.rn.f16x2 h0, h0, %9, %13;\n\t"
         "fma.rn.f16x2 h1, h1, %9, %13;\n\t"
         "fma.rn.f16x2 h2, h2, %10, %14;\n\t"
@@ -564,8 +616,10 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
         "}\n"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
         : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(0x38003800u), "r"(0x30003000u),
-          "r"(0x28002800u), "r"(0x20002000u), "r"(0xE006E006u), "r"(0xD818D818u),
-          "r"(0xD060D060u), "r"(0xC980C980u));
+          "r"(0x28002800u), "r"(0x20002000u), "r"(kBits == 2 ? 0xE006E006u : 0xE002E002u),
+          "r"(kBits == 2 ? 0xD818D818u : 0xD808D808u), "r"(kBits == 2 ? 0xD060D060u : 0xD020D020u),
+          "r"(kBits == 2 ? 0xC980C980u : 0xC880C880u), "n"(dq_mask<kBits>(0)),
+          "n"(dq_mask<kBits>(1)), "n"(dq_mask<kBits>(2)), "n"(dq_mask<kBits>(3)));
 }
 
 // The same block without normalising the codes: each fragment register holds
@@ -578,6 +632,7 @@ STRATA_DEV void block_mma2(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, 
 // result is 2^8 sum_k (q_k - 1.5) x_k, the block's dot product with the
 // dequantised weights over its scale, times 2^8.  Two shifts and 8 mask/or
 // per block, no packed fma.
+template <int kBits = 2>
 STRATA_DEV void block_mma2m(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1, uint32_t b2,
                             uint32_t b3, float c0, float c1) {
     asm(
@@ -585,31 +640,33 @@ STRATA_DEV void block_mma2m(float (&d)[4], uint32_t w, uint32_t b0, uint32_t b1,
         ".reg .b32 s8, s2, h0, h1, h2, h3, h4, h5, h6, h7;\n\t"
         "shr.b32 s8, %4, 8;\n\t"
         "shl.b32 s2, %4, 8;\n\t"
-        "lop3.b32 h0, %4, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h1, s8, 0x000C000C, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h2, %4, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h3, s8, 0x00300030, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h4, %4, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h5, s8, 0x00C000C0, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h6, %4, 0x03000300, 0x64006400, 0xEA;\n\t"
-        "lop3.b32 h7, s2, 0x03000300, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h0, %4, %11, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h1, s8, %11, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h2, %4, %12, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h3, s8, %12, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h4, %4, %13, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h5, s8, %13, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h6, %4, %14, 0x64006400, 0xEA;\n\t"
+        "lop3.b32 h7, s2, %14, 0x64006400, 0xEA;\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h0,h1,h2,h3}, "
         "{%5,%6}, {%9,%10,%9,%10};\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {h4,h5,h6,h7}, "
         "{%7,%8}, {%0,%1,%2,%3};\n\t"
         "}\n"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "f"(c0), "f"(c1));
+        : "r"(w), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "f"(c0), "f"(c1), "n"(dq_mask<kBits>(0)),
+          "n"(dq_mask<kBits>(1)), "n"(dq_mask<kBits>(2)), "n"(dq_mask<kBits>(3)));
 }
 
 // Column factor of the magic-offset token operand and the correction weight
 // of column k of a block (see block_mma2m), kk = k mod 32:
-// B_k = x_k * magic_col_scale(kk) = x_k 2^(8 - P_k), c_k = 1024 + 1.5 * 2^P_k.
+// B_k = x_k * magic_col_scale(kk) = x_k 2^(8 - P_k), c_k = 1024 + centre 2^P_k.
 __host__ __device__ inline float magic_col_scale(int kk) {  // kk = k mod 32
     return (float)(1 << (6 - 2 * (kk >> 3)));
 }
-__host__ __device__ inline float magic_col_corr(int kk) {
-    return 1024.0f + 1.5f * (float)(1 << (2 + 2 * (kk >> 3)));
+__host__ __device__ inline float magic_col_corr(int kk, int bits = 2) {
+    // 1024 + centre 2^P_k, centre = (2^bits - 1) / 2 (1.5 for 2-bit, 0.5 for 1-bit)
+    return 1024.0f + 0.5f * (float)((1 << bits) - 1) * (float)(1 << (2 + 2 * (kk >> 3)));
 }
 
 // ---------------------------------------------------------------- GEMV blocks

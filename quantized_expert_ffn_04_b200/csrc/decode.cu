@@ -224,9 +224,9 @@ template <int kBits, bool kMagic>
 STRATA_DEV void block_dot(float (&d)[4], uint32_t lo, uint32_t hi, int hshift, uint32_t b0,
                           uint32_t b1, uint32_t b2, uint32_t b3, float c0, float c1) {
     if (kMagic)
-        block_mma2m(d, lo, b0, b1, b2, b3, c0, c1);
-    else if (kBits == 2)
-        block_mma2(d, lo, b0, b1, b2, b3);
+        block_mma2m<kBits>(d, lo, b0, b1, b2, b3, c0, c1);
+    else if (kBits <= 2)
+        block_mma2<kBits>(d, lo, b0, b1, b2, b3);
     else
         block_mma<kBits>(d, lo, hi, hshift, b0, b1, b2, b3);
 }
@@ -247,7 +247,7 @@ STRATA_DEV void slab2_blocks(float (&acc0)[4], float (&acc1)[4], const uint8_t *
                              const uint8_t *s1, int b0, int b1, const __half *rowp,
                              const float *ca, const float *cb, int lane) {
     constexpr int UB = unit_bytes(kBits);
-    constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
+    constexpr int SOFF = scale_off(kBits);
     const int g = lane >> 2;
     int b = b0;
     for (; b + 4 <= b1; b += 4) {
@@ -257,8 +257,15 @@ STRATA_DEV void slab2_blocks(float (&acc0)[4], float (&acc1)[4], const uint8_t *
         for (int pp = 0; pp < 2; pp++) {
             const int bp = b + 2 * pp;
             const int off = (bp >> 2) * UB, wo = (bp & 3) * 4;
-            lw[pp][0] = *reinterpret_cast<const uint2 *>(s0 + off + lane * 16 + wo);
-            lw[pp][1] = *reinterpret_cast<const uint2 *>(s1 + off + lane * 16 + wo);
+            if (kBits == 1) {  // one word, both blocks of the pair (odd one a bit higher)
+                const uint32_t v0 = *reinterpret_cast<const uint32_t *>(s0 + off + lane * 8 + wo / 2);
+                const uint32_t v1 = *reinterpret_cast<const uint32_t *>(s1 + off + lane * 8 + wo / 2);
+                lw[pp][0] = make_uint2(v0, v0 >> 1);
+                lw[pp][1] = make_uint2(v1, v1 >> 1);
+            } else {
+                lw[pp][0] = *reinterpret_cast<const uint2 *>(s0 + off + lane * 16 + wo);
+                lw[pp][1] = *reinterpret_cast<const uint2 *>(s1 + off + lane * 16 + wo);
+            }
             kw[pp][0] = *reinterpret_cast<const uint2 *>(s0 + off + SOFF + g * 16 + wo);
             kw[pp][1] = *reinterpret_cast<const uint2 *>(s1 + off + SOFF + g * 16 + wo);
             if (kBits == 3) {
@@ -297,8 +304,8 @@ STRATA_DEV void slab2_blocks(float (&acc0)[4], float (&acc1)[4], const uint8_t *
     for (; b < b1; b++) {
         const uint8_t *u0 = s0 + (b >> 2) * UB, *u1 = s1 + (b >> 2) * UB;
         const int blk = b & 3;
-        const uint32_t lw0 = *reinterpret_cast<const uint32_t *>(u0 + lane * 16 + blk * 4);
-        const uint32_t lw1 = *reinterpret_cast<const uint32_t *>(u1 + lane * 16 + blk * 4);
+        const uint32_t lw0 = unit_word<kBits>(u0, lane, blk);
+        const uint32_t lw1 = unit_word<kBits>(u1, lane, blk);
         const uint32_t kw0 = *reinterpret_cast<const uint32_t *>(u0 + SOFF + g * 16 + blk * 4);
         const uint32_t kw1 = *reinterpret_cast<const uint32_t *>(u1 + SOFF + g * 16 + blk * 4);
         uint32_t hw0 = 0, hw1 = 0;
@@ -393,14 +400,14 @@ STRATA_DEV bool grid_barrier(unsigned long long *bar, unsigned long long target,
 template <int kBits>
 STRATA_DEV __half token_operand(float x, int ex, int i) {
     const float v = x * pow2f(-ex);
-    return __float2half_rn(kBits == 2 ? v * magic_col_scale(i & 31) : v);
+    return __float2half_rn(kBits <= 2 ? v * magic_col_scale(i & 31) : v);
 }
 template <int kBits>
 STRATA_DEV float block_correction(const __nv_bfloat16 *blk, int ex) {
     float v = 0.0f;
 #pragma unroll 8
     for (int kk = 0; kk < 32; kk++)
-        v = fmaf(-magic_col_corr(kk),
+        v = fmaf(-magic_col_corr(kk, kBits),
                  __half2float(token_operand<kBits>(__bfloat162float(blk[kk]), ex, kk)), v);
     return v;
 }
@@ -419,7 +426,7 @@ template <int kBits, bool kStaged>
 __device__ __noinline__ int fused_run_items(const FusedParams &p, int jpos, int stop) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int UB = unit_bytes(kBits);
-    constexpr bool kMagic = kBits == 2;
+    constexpr bool kMagic = kBits <= 2;  // magic-offset gate/up (1- and 2-bit)
     constexpr bool staged = kStaged;
     const FusedSmem L = fused_smem(p.T, p.E, p.k, p.H, p.Ip, p.ring, p.item_bytes, p.staged,
                                    p.units_max, p.na);
@@ -626,7 +633,7 @@ template <int kBits, bool kStaged>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int UB = unit_bytes(kBits);
-    constexpr bool kMagic = kBits == 2;
+    constexpr bool kMagic = kBits <= 2;  // magic-offset gate/up (1- and 2-bit)
     const FusedSmem L = fused_smem(p.T, p.E, p.k, p.H, p.Ip, p.ring, p.item_bytes, p.staged,
                                    p.units_max, p.na);
     uint8_t *ring = sm + L.ring;
@@ -952,29 +959,51 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                     ready &= ready - 1;
                     const int tt = __shfl_sync(0xffffffffu, t, j);
                     const int ex = staged ? sex[tt] : __ldcg(p.xex + tt);
+                    // lane: 4 adjacent columns of the 128-row block, every
+                    // row one 16-byte load; the loads are unconditional (picks
+                    // past k re-read the last one and add an exact zero with
+                    // weight 0), so all k + 1 rows are in flight at once
+                    const int col = part * kSlabRows * kDownSlabs + 4 * lane;
+                    const int *so = sord + tt * k;
+                    float4 vv[kFMaxK];
 #pragma unroll
-                    for (int cc = 0; cc < 4; cc++) {
-                        const int col = part * kSlabRows * kDownSlabs + cc * 32 + lane;
-                        // unconditional loads (picks past k re-read the last
-                        // one): all k + 1 rows are in flight at once
-                        float vv[kFMaxK];
+                    for (int r = 0; r < kFMaxK; r++)
+                        vv[r] = __ldcg(reinterpret_cast<const float4 *>(
+                            p.Y + (size_t)sslot[so[r < k ? r : k - 1]] * H + col));
+                    float4 acc = __ldcg(reinterpret_cast<const float4 *>(p.Y + (size_t)(Tk + tt) * H + col));
 #pragma unroll
-                        for (int r = 0; r < kFMaxK; r++)
-                            vv[r] = __ldcg(p.Y + (size_t)sslot[sord[tt * k + (r < k ? r : k - 1)]] * H + col);
-                        float acc2 = __ldcg(p.Y + (size_t)(Tk + tt) * H + col);
-                        // picks past k add an exact zero (weight 0, a finite
-                        // row), so every load is used and none is sunk into a
-                        // branch
-#pragma unroll
-                        for (int r = 0; r < kFMaxK; r++)
-                            acc2 = fmaf(r < k ? sw[sord[tt * k + r]] : 0.0f, vv[r], acc2);
-                        if (ex) acc2 = acc2 * pow2f(ex) * pow2f(ex);
-                        __nv_bfloat16 *o = p.out + (size_t)tt * H + col;
-                        const __nv_bfloat16 yb = __float2bfloat16_rn(acc2);
-                        *o = p.residual ? __float2bfloat16_rn(__fadd_rn(__bfloat162float(*o),
-                                                                        __bfloat162float(yb)))
-                                        : yb;
+                    for (int r = 0; r < kFMaxK; r++) {
+                        const float wr = r < k ? sw[so[r]] : 0.0f;
+                        acc.x = fmaf(wr, vv[r].x, acc.x);
+                        acc.y = fmaf(wr, vv[r].y, acc.y);
+                        acc.z = fmaf(wr, vv[r].z, acc.z);
+                        acc.w = fmaf(wr, vv[r].w, acc.w);
                     }
+                    if (ex) {  // the token's prescale off (2^ex twice: stays in range)
+                        const float f = pow2f(ex);
+                        acc.x = acc.x * f * f;
+                        acc.y = acc.y * f * f;
+                        acc.z = acc.z * f * f;
+                        acc.w = acc.w * f * f;
+                    }
+                    __nv_bfloat16 *o = p.out + (size_t)tt * H + col;
+                    __nv_bfloat162 y01 = __floats2bfloat162_rn(acc.x, acc.y);
+                    __nv_bfloat162 y23 = __floats2bfloat162_rn(acc.z, acc.w);
+                    if (p.residual) {
+                        const uint2 hv = *reinterpret_cast<const uint2 *>(o);
+                        const __nv_bfloat162 h01 = *reinterpret_cast<const __nv_bfloat162 *>(&hv.x);
+                        const __nv_bfloat162 h23 = *reinterpret_cast<const __nv_bfloat162 *>(&hv.y);
+                        y01 = __floats2bfloat162_rn(
+                            __fadd_rn(__low2float(h01), __low2float(y01)),
+                            __fadd_rn(__high2float(h01), __high2float(y01)));
+                        y23 = __floats2bfloat162_rn(
+                            __fadd_rn(__low2float(h23), __low2float(y23)),
+                            __fadd_rn(__high2float(h23), __high2float(y23)));
+                    }
+                    uint2 ov;
+                    ov.x = *reinterpret_cast<const uint32_t *>(&y01);
+                    ov.y = *reinterpret_cast<const uint32_t *>(&y23);
+                    *reinterpret_cast<uint2 *>(o) = ov;
                 }
             }
             __syncwarp();
@@ -1343,8 +1372,9 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     const int nwc = (wb + p.item_bytes - 1) / p.item_bytes;
     if (p.ring < 2 || nwc >= p.ring) return cudaErrorInvalidValue;
     const int smem = total(p.ring, p.staged, p.na);
-    auto kern = g.bits == 2 ? (p.staged ? fused_decode_kernel<2, true> : fused_decode_kernel<2, false>)
-                            : (p.staged ? fused_decode_kernel<3, true> : fused_decode_kernel<3, false>);
+    auto kern = g.bits == 1   ? (p.staged ? fused_decode_kernel<1, true> : fused_decode_kernel<1, false>)
+                : g.bits == 2 ? (p.staged ? fused_decode_kernel<2, true> : fused_decode_kernel<2, false>)
+                              : (p.staged ? fused_decode_kernel<3, true> : fused_decode_kernel<3, false>);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kFThreads);
@@ -1365,6 +1395,8 @@ cudaError_t fused_init_attributes(int max_smem) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&g_fused_sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<1, true>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(fused_decode_kernel<1, false>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(fused_decode_kernel<2, true>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(fused_decode_kernel<2, false>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(fused_decode_kernel<3, true>, max_smem)) != cudaSuccess) return e;

@@ -14,7 +14,8 @@
 //   -> all-to-all of the outputs back, in the same order -> the home rank runs
 //   the shared expert and combines in the layer's fixed order.
 // Each expert output is a function of one token row and one expert only, so
-// the result is the same bits as on one GPU whatever the batch around it.
+// the result is the same bits as on one GPU on the same kernels, whatever the
+// batch around it.
 #include <cuda_runtime.h>
 
 #include <vector>

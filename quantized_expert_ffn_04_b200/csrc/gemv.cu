@@ -35,11 +35,17 @@ template <int kBits>
 __device__ __forceinline__ void slab_dot(float (&acc)[4], const uint8_t *w, int ns,
                                          const uint16_t *xb, int pitch, int xrows, int lane) {
     constexpr int UB = unit_bytes(kBits);
-    constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
+    constexpr int SOFF = scale_off(kBits);
     const uint16_t *xrow = xb + ((lane & 7) < xrows ? (lane & 7) : 0) * pitch;
     for (int sg = 0; sg < ns; sg++) {
         const uint8_t *un = w + sg * UB;
-        uint4 lo = *reinterpret_cast<const uint4 *>(un + lane * 16);
+        uint4 lo;
+        if (kBits == 1) {  // two words, two blocks each (the odd block one bit higher)
+            const uint2 v = *reinterpret_cast<const uint2 *>(un + lane * 8);
+            lo = make_uint4(v.x, v.x >> 1, v.y, v.y >> 1);
+        } else {
+            lo = *reinterpret_cast<const uint4 *>(un + lane * 16);
+        }
         uint2 hi = make_uint2(0, 0);
         if (kBits == 3) hi = *reinterpret_cast<const uint2 *>(un + kLoBytes + lane * 8);
         uint32_t sc = *reinterpret_cast<const uint32_t *>(un + SOFF + lane * 4);
@@ -49,8 +55,8 @@ __device__ __forceinline__ void slab_dot(float (&acc)[4], const uint8_t *w, int 
             ldmatrix_x4(b0, b1, b2, b3, xrow + sg * 128 + blk * 32 + (lane >> 3) * 8);
             uint32_t s2 = __shfl_sync(0xffffffffu, sc, (lane & ~3) | blk);
             float d[4];
-            if (kBits == 2)
-                block_mma2(d, comp4(lo, blk), b0, b1, b2, b3);
+            if (kBits <= 2)
+                block_mma2<kBits>(d, comp4(lo, blk), b0, b1, b2, b3);
             else
                 block_mma<kBits>(d, comp4(lo, blk), blk < 2 ? hi.x : hi.y, 8 * (blk & 1), b0, b1,
                                  b2, b3);
@@ -147,19 +153,22 @@ __global__ __launch_bounds__(128) void gemv_gateup_kernel(
             }
 #pragma unroll
             for (int b = 0; b < 8; b++) {
+                // every lane takes part in the shuffle (no lane leaves the
+                // loop early), then only the lanes with a chunk store it
                 const int idx = base + b * 32 + lane;
                 const int j = idx / per_row, i = idx % per_row;
                 const float sc = pow2f(-__shfl_sync(0xffffffffu, my_ex, j & 31));
-                if (idx >= nchunk) break;
-                const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&v[b]);
-                uint4 o;
-                __half2 *h = reinterpret_cast<__half2 *>(&o);
+                if (idx < nchunk) {
+                    const __nv_bfloat162 *bb = reinterpret_cast<const __nv_bfloat162 *>(&v[b]);
+                    uint4 o;
+                    __half2 *h = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    const float2 f = __bfloat1622float2(bb[q]);
-                    h[q] = __floats2half2_rn(f.x * sc, f.y * sc);
+                    for (int q = 0; q < 4; q++) {
+                        const float2 f = __bfloat1622float2(bb[q]);
+                        h[q] = __floats2half2_rn(f.x * sc, f.y * sc);
+                    }
+                    reinterpret_cast<uint4 *>(xb + j * pitch)[i] = o;
                 }
-                reinterpret_cast<uint4 *>(xb + j * pitch)[i] = o;
             }
         }
     }
@@ -287,7 +296,8 @@ void launch_gemv_gateup(const Geometry &g, const ExpertWeights &w, const int4 *u
     dim3 grid((unsigned)((size_t)units_max * (g.Ip / kSlabRows)));
     auto xb = reinterpret_cast<const __nv_bfloat16 *>(x);
     auto ao = reinterpret_cast<__half *>(a_out);
-    auto kern = g.bits == 2 ? gemv_gateup_kernel<2> : gemv_gateup_kernel<3>;
+    auto kern = g.bits == 1 ? gemv_gateup_kernel<1>
+                : g.bits == 2 ? gemv_gateup_kernel<2> : gemv_gateup_kernel<3>;
     launch_pdl(kern, grid, dim3(128), smem, s, w.routed, w.shared, g.expert_bytes, g.mat_bytes,
                units, n_units, list, Tk, T, g.E, xb, xex, g.H, g.Ip, xrows, nsh,
                shared_rows < 0 ? T : shared_rows, ao, err, budget);
@@ -300,13 +310,16 @@ void launch_gemv_down(const Geometry &g, const ExpertWeights &w, const int4 *uni
     size_t smem = down_smem(g, xrows);
     dim3 grid((unsigned)((size_t)units_max * (g.H / 64)));
     auto ap = reinterpret_cast<const __half *>(a);
-    auto kern = g.bits == 2 ? gemv_down_kernel<2> : gemv_down_kernel<3>;
+    auto kern = g.bits == 1 ? gemv_down_kernel<1>
+                : g.bits == 2 ? gemv_down_kernel<2> : gemv_down_kernel<3>;
     launch_pdl(kern, grid, dim3(128), smem, s, w.routed, w.shared, g.expert_bytes, g.mat_bytes,
                units, n_units, g.E, ap, g.H, g.Ip, xrows, Y, err, budget);
 }
 
 cudaError_t gemv_init_attributes(int max_smem) {
     cudaError_t e;
+    if ((e = allow_max_dyn_smem(gemv_gateup_kernel<1>, max_smem)) != cudaSuccess) return e;
+    if ((e = allow_max_dyn_smem(gemv_down_kernel<1>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(gemv_gateup_kernel<2>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(gemv_gateup_kernel<3>, max_smem)) != cudaSuccess) return e;
     if ((e = allow_max_dyn_smem(gemv_down_kernel<2>, max_smem)) != cudaSuccess) return e;

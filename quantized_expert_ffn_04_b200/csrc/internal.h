@@ -78,6 +78,11 @@ void launch_route_small(const float *logits, int T, int E, int k, int32_t *idx, 
 void launch_screen_topk(const float *D, int R, const void *x, int T, int H, const float *Wp,
                         const float *bias, int E, int k, float gam, float wmax, float bmax,
                         int32_t *idx, float *w, cudaStream_t s);
+// Test hook: the screen's approximate logits a [T][E] (the two split-GEMM
+// columns plus the bias) and each token's eps (0: not covered by the bound).
+void launch_screen_debug(const float *D, int R, const void *x, int T, int H, const float *bias,
+                         int E, float gam, float wmax, float bmax, float *a_out, float *eps_out,
+                         cudaStream_t s);
 
 // ---- gemv.cu (decode)
 struct ExpertWeights {

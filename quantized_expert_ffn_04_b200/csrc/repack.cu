@@ -45,7 +45,7 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes,
             for (int half = 0; half < 2; half++) {
                 int col = col0 + half;
                 int q = (row < R && col < K) ? canon_code(codes, bits, K, row, col) : 0;
-                lo[w] |= (uint32_t)(q & 3) << (code_pos(bits, rp) + 16 * half);
+                lo[w] |= (uint32_t)(q & 3) << (code_pos(bits == 1 ? 2 : bits, rp) + 16 * half);
                 if (bits == 3)
                     hi[w >> 1] |= (uint32_t)((q >> 2) & 1) << (rp + 8 * (w & 1) + 16 * half);
             }
@@ -57,8 +57,11 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes,
         int blkcol = seg * 4 + c;
         sc[h] = (row < R && blkcol * 32 < K) ? scales[(size_t)row * (K / 32) + blkcol] : 0;
     }
-    reinterpret_cast<uint4 *>(u)[lane] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    int off = kLoBytes;
+    if (bits == 1)  // blocks 2h and 2h + 1 share word h, the odd one a bit higher
+        reinterpret_cast<uint2 *>(u)[lane] = make_uint2(lo[0] | (lo[1] << 1), lo[2] | (lo[3] << 1));
+    else
+        reinterpret_cast<uint4 *>(u)[lane] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    int off = lo_bytes(bits);
     if (bits == 3) {
         reinterpret_cast<uint2 *>(u + off)[lane] = make_uint2(hi[0], hi[1]);
         off += kHiBytes;
@@ -117,9 +120,9 @@ __device__ float debug_weight(const uint8_t *mat, int Kp, int row, int col, int 
     int c = (kk & 7) >> 1, half = kk & 1;
     int lane = 4 * g + c;
     int rp = 4 * s + r;
-    uint32_t lo = reinterpret_cast<const uint32_t *>(u)[lane * 4 + w];
+    uint32_t lo = unit_word<kBits>(u, lane, w);
     uint32_t hi = 0;
-    int off = kLoBytes;
+    int off = lo_bytes(kBits);
     if (kBits == 3) {
         hi = reinterpret_cast<const uint32_t *>(u + off)[lane * 2 + (w >> 1)];
         off += kHiBytes;
@@ -130,13 +133,14 @@ __device__ float debug_weight(const uint8_t *mat, int Kp, int row, int col, int 
     __half d = __ushort_as_half(dbits);
     if (kind == 0) {
         // the code read straight from its bit position, then 2q - (2^bits - 1)
-        int q = (lo >> (code_pos(kBits, rp) + 16 * half)) & 3;
+        int q = (lo >> (code_pos(kBits == 1 ? 2 : kBits, rp) + 16 * half)) & (kBits == 1 ? 1 : 3);
         if (kBits == 3) q |= ((hi >> (rp + 8 * (w & 1) + 16 * half)) & 1) << 2;
         const float q2 = (float)(2 * q - ((1 << kBits) - 1));
         return q2 * (__half2float(d) * 0.5f);  // exact in fp32
     } else {
         // the tensor-core operand, computed by the prefill kernels' routine
-        uint32_t p = kBits == 2 ? dq2_pair(lo, rp) : dq_pair<false, kBits>(lo, hi, rp, 8 * (w & 1));
+        uint32_t p = kBits <= 2 ? dq2_pair<kBits == 1 ? 1 : 2>(lo, rp)
+                                : dq_pair<false, kBits>(lo, hi, rp, 8 * (w & 1));
         __half2 v = *reinterpret_cast<__half2 *>(&p);
         __half dh = __hmul(d, __float2half(0.5f));
         __half2 wv = __hmul2(v, __half2half2(dh));
@@ -149,8 +153,9 @@ __global__ void debug_dequant_kernel(const uint8_t *mat, int bits, int Kp, int r
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)nrows * ncols) return;
     int r = (int)(i / ncols), c = (int)(i % ncols);
-    out[i] = bits == 2 ? debug_weight<2>(mat, Kp, row0 + r, c, kind)
-                       : debug_weight<3>(mat, Kp, row0 + r, c, kind);
+    out[i] = bits == 1   ? debug_weight<1>(mat, Kp, row0 + r, c, kind)
+             : bits == 2 ? debug_weight<2>(mat, Kp, row0 + r, c, kind)
+                         : debug_weight<3>(mat, Kp, row0 + r, c, kind);
 }
 
 void launch_debug_dequant(const uint8_t *mat, int bits, int Kp, int row0, int nrows, int ncols,

@@ -431,6 +431,64 @@ void launch_dispatch(const int32_t *idx, int T, int k, int E, int32_t *cnt, int3
 // below, adding 2^-25 ||W_e||_1 <= 2^-25 sqrt(H) ||W_e||_2; a token with any
 // |x| > 65504 (or a non-finite bound) keeps every expert as a candidate.
 
+// The screening bound of one token (one warp; see above): the token row's
+// L2 norm, L1 norm and largest magnitude, and eps from them.  When xs is not
+// NULL the row is also stored there in the router's lane-interleaved fp32
+// layout.  `finite` is false for a token the bound does not cover (a
+// non-finite bound, or an entry beyond fp16's range).
+__device__ float screen_eps(const __nv_bfloat16 *__restrict__ xr, int H, float gam, float wmax,
+                            float bmax, int lane, float4 *xs, bool &finite) {
+    const int ns4 = H / 128;
+    float ss = 0.f, s1 = 0.f, xm = 0.f;
+    for (int s4 = 0; s4 < ns4; s4++) {
+        float v0 = __bfloat162float(xr[128 * s4 + lane]);
+        float v1 = __bfloat162float(xr[128 * s4 + 32 + lane]);
+        float v2 = __bfloat162float(xr[128 * s4 + 64 + lane]);
+        float v3 = __bfloat162float(xr[128 * s4 + 96 + lane]);
+        ss = fmaf(v0, v0, fmaf(v1, v1, fmaf(v2, v2, fmaf(v3, v3, ss))));
+        s1 += fabsf(v0) + fabsf(v1) + fabsf(v2) + fabsf(v3);
+        xm = fmaxf(xm, fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+        if (xs) xs[s4 * 32 + lane] = make_float4(v0, v1, v2, v3);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, o));
+    }
+    __syncwarp();
+    const float eps =
+        2.0f * (gam * sqrtf(ss) * 1.001f * wmax + 2.9802322e-8f * s1 * 1.001f +
+                2.9802322e-8f * sqrtf((float)H) * wmax + 2.3841858e-7f * bmax);
+    finite = isfinite(eps) && !(xm > 65504.0f);
+    return eps;
+}
+
+// Test hook: the approximate logits a[t][e] the screen compares and each
+// token's eps (0 when the bound does not cover the token).  One warp per token.
+__global__ void screen_debug_kernel(const float *__restrict__ D, int R,
+                                    const __nv_bfloat16 *__restrict__ x, int T, int H,
+                                    const float *__restrict__ bias, int E, float gam, float wmax,
+                                    float bmax, float *__restrict__ a_out,
+                                    float *__restrict__ eps_out) {
+    const int t = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= T) return;
+    bool finite;
+    const float eps = screen_eps(x + (size_t)t * H, H, gam, wmax, bmax, lane, nullptr, finite);
+    if (lane == 0) eps_out[t] = finite ? eps : 0.0f;
+    const float *dr = D + (size_t)t * R;
+    for (int e = lane; e < E; e += 32)
+        a_out[(size_t)t * E + e] = (dr[e] + dr[E + e]) + (bias ? bias[e] : 0.0f);
+}
+
+void launch_screen_debug(const float *D, int R, const void *x, int T, int H, const float *bias,
+                         int E, float gam, float wmax, float bmax, float *a_out, float *eps_out,
+                         cudaStream_t s) {
+    screen_debug_kernel<<<(T + 3) / 4, 128, 0, s>>>(
+        D, R, reinterpret_cast<const __nv_bfloat16 *>(x), T, H, bias, E, gam, wmax, bmax, a_out,
+        eps_out);
+}
+
 // k picks among the lanes' values v (lane l holds experts l, l+32, ...);
 // experts whose bit is set in `taken` are excluded.  Lane j < k ends with pick
 // j; writes idx/w.
@@ -488,42 +546,19 @@ __global__ __launch_bounds__(128) void screen_topk_kernel(
     const int ns4 = H / 128;
     float4 *xs = sm4 + (size_t)warp * (H / 4);
     float *exl = reinterpret_cast<float *>(sm4 + 4 * (H / 4)) + warp * 1024;
-    // token row in the router's lane-interleaved fp32 layout, and its norms
-    float ss = 0.f, s1 = 0.f, xm = 0.f;
-    const __nv_bfloat16 *xr = x + (size_t)t * H;
-    for (int s4 = 0; s4 < ns4; s4++) {
-        float v0 = __bfloat162float(xr[128 * s4 + lane]);
-        float v1 = __bfloat162float(xr[128 * s4 + 32 + lane]);
-        float v2 = __bfloat162float(xr[128 * s4 + 64 + lane]);
-        float v3 = __bfloat162float(xr[128 * s4 + 96 + lane]);
-        ss = fmaf(v0, v0, fmaf(v1, v1, fmaf(v2, v2, fmaf(v3, v3, ss))));
-        s1 += fabsf(v0) + fabsf(v1) + fabsf(v2) + fabsf(v3);
-        xm = fmaxf(xm, fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
-        xs[s4 * 32 + lane] = make_float4(v0, v1, v2, v3);
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, o));
-    }
-    __syncwarp();
-    const float eps =
-        2.0f * (gam * sqrtf(ss) * 1.001f * wmax + 2.9802322e-8f * s1 * 1.001f +
-                2.9802322e-8f * sqrtf((float)H) * wmax + 2.3841858e-7f * bmax);
-    const bool finite = isfinite(eps) && !(xm > 65504.0f);
+    bool finite;
+    const float eps = screen_eps(x + (size_t)t * H, H, gam, wmax, bmax, lane, xs, finite);
     const int nq = (E + 31) >> 5;
     const float *dr = D + (size_t)t * R;
     float av[32];
+    // unconditional loads (entries past E re-read expert 0), so the compiler
+    // cannot sink them into branches and issue them one by one
 #pragma unroll
     for (int q = 0; q < 32; q++) {
-        int e = q * 32 + lane;
-        float a = -INFINITY;
-        if (q < nq && e < E) {
-            a = (dr[e] + dr[E + e]) + (bias ? bias[e] : 0.0f);
-            if (a != a) a = INFINITY;  // keep a NaN screening value as a candidate
-        }
-        av[q] = a;
+        const int e = q * 32 + lane, ec = e < E ? e : 0;
+        float a = (dr[ec] + dr[E + ec]) + (bias ? bias[ec] : 0.0f);
+        if (a != a) a = INFINITY;  // keep a NaN screening value as a candidate
+        av[q] = (q < nq && e < E) ? a : -INFINITY;
     }
     // k-th largest approximate logit
     uint32_t taken = 0;

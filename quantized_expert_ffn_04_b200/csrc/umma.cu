@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
             const int L = dt & 31, sl0 = dt >> 5;        // slabs sl0 and sl0 + 4
             const int g8 = L >> 2, c = L & 3;
             constexpr int UB = unit_bytes(kBits);
-            constexpr int SOFF = kLoBytes + (kBits == 3 ? kHiBytes : 0);
+            constexpr int SOFF = scale_off(kBits);
             const __half2 half2_05 = __float2half2_rn(0.5f);
             // packed words of one stage for this thread: [matrix][slab]
             struct Raw {
@@ -304,7 +304,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                     for (int si = 0; si < 2; si++) {
                         const uint8_t *un = wbase + m * p.mat_bytes +
                                             ((size_t)(rt * 8 + sl0 + 4 * si) * p.nseg + seg) * UB;
-                        r.lo[m][si] = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
+                        if (kBits == 1) {  // blocks 2h, 2h + 1 in one word (the odd one a bit higher)
+                            const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(un + L * 8 + 4 * h));
+                            r.lo[m][si] = make_uint2(v, v >> 1);
+                        } else {
+                            r.lo[m][si] = __ldg(reinterpret_cast<const uint2 *>(un + L * 16 + 8 * h));
+                        }
                         r.hi[m][si] = kBits == 3 ? __ldg(reinterpret_cast<const uint32_t *>(
                                                        un + kLoBytes + L * 8 + 4 * h))
                                                  : 0u;
@@ -349,7 +354,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
 #pragma unroll
                                 for (int r = 0; r < 4; r++) {
                                     const uint32_t pr =
-                                        kBits == 2 ? dq2_pair(lw, 4 * s + r)
+                                        kBits <= 2 ? dq2_pair<kBits == 1 ? 1 : 2>(lw, 4 * s + r)
                                                    : dq_pair<false, kBits>(lw, cur.hi[m][si],
                                                                            4 * s + r, 8 * bw);
                                     const __half2 v = __hmul2(u2h(pr), (r & 1) ? s_hi : s_lo);
@@ -616,8 +621,9 @@ cudaError_t launch_umma_gateup(const Geometry &g, const ExpertWeights &w, const 
     p.n_rt = g.Ip / kTM;
     p.out = reinterpret_cast<__half *>(a);
     p.out_ld = g.Ip;
-    return g.bits == 2 ? run_umma<2, kModeGateUp>(p, units_max * p.n_rt, s)
-                       : run_umma<3, kModeGateUp>(p, units_max * p.n_rt, s);
+    return g.bits == 1   ? run_umma<1, kModeGateUp>(p, units_max * p.n_rt, s)
+           : g.bits == 2 ? run_umma<2, kModeGateUp>(p, units_max * p.n_rt, s)
+                         : run_umma<3, kModeGateUp>(p, units_max * p.n_rt, s);
 }
 
 cudaError_t launch_umma_down(const Geometry &g, const ExpertWeights &w, const int4 *units,
@@ -633,8 +639,9 @@ cudaError_t launch_umma_down(const Geometry &g, const ExpertWeights &w, const in
     p.n_rt = g.H / kTM;
     p.out = reinterpret_cast<__half *>(Y);
     p.out_ld = g.H;
-    return g.bits == 2 ? run_umma<2, kModeDown>(p, units_max * p.n_rt, s)
-                       : run_umma<3, kModeDown>(p, units_max * p.n_rt, s);
+    return g.bits == 1   ? run_umma<1, kModeDown>(p, units_max * p.n_rt, s)
+           : g.bits == 2 ? run_umma<2, kModeDown>(p, units_max * p.n_rt, s)
+                         : run_umma<3, kModeDown>(p, units_max * p.n_rt, s);
 }
 
 cudaError_t launch_umma_plain(const __half *A, int rows, const __half *x16, int T, int K, float *D,
@@ -658,6 +665,10 @@ cudaError_t umma_init_attributes(int max_smem) {
     // look the encoder up here, outside any stream capture
     if (!encode_fn()) return cudaErrorNotSupported;
     cudaError_t e;
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<1, kModeGateUp>, max_smem)) != cudaSuccess)
+        return e;
+    if ((e = allow_max_dyn_smem(umma_expert_kernel<1, kModeDown>, max_smem)) != cudaSuccess)
+        return e;
     if ((e = allow_max_dyn_smem(umma_expert_kernel<2, kModeGateUp>, max_smem)) != cudaSuccess)
         return e;
     if ((e = allow_max_dyn_smem(umma_expert_kernel<3, kModeGateUp>, max_smem)) != cudaSuccess)

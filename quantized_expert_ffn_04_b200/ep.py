@@ -16,7 +16,10 @@ the router and the shared expert.  A forward of the rank's own T tokens:
 
 Each expert output depends on one token row and one expert only, and the
 combine is the one-GPU combine on the same values, so the result is the same
-bits as the one-GPU forward of the rank's tokens.  The exchange is
+bits as the one-GPU forward of the rank's tokens on the same kernels (the
+decode GEMV chain up to 64 tokens, the tensor-core prefill above; the fused
+decode kernel sums its K partials in another order and agrees within the
+layer tolerance).  The exchange is
 torch.distributed's all_to_all_single (NCCL on GPUs, gloo on CPU).
 
 The compute steps go through a backend; GpuBackend calls the library's

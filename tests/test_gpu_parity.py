@@ -69,6 +69,10 @@ CASES = [
     ("flash3-T64", gen.FLASH3, 64),
     ("pruned256-T4", gen.PRUNED256, 4),
     ("pruned256-T300", gen.PRUNED256, 300),
+    ("tiny1-T8", gen.TINY1, 8),
+    ("coder1-T4", gen.CODER1, 4),
+    ("coder1-T13", gen.CODER1, 13),
+    ("coder1-T300", gen.CODER1, 300),
 ]
 
 
@@ -84,7 +88,8 @@ def test_route_and_forward_parity(name, shape, T):
     check_output(y, ref, name)
 
 
-@pytest.mark.parametrize("shape", [gen.TINY, gen.FLASH2, gen.FLASH3], ids=["tiny", "f2", "f3"])
+@pytest.mark.parametrize("shape", [gen.TINY, gen.FLASH2, gen.FLASH3, gen.CODER1],
+                         ids=["tiny", "f2", "f3", "c1"])
 def test_dequant_bit_exact(shape):
     w = layer_of(shape)
     L = gpu_layer(shape, 1)
@@ -133,6 +138,8 @@ PATH_CASES = [
     ("f2-T65-auto", gen.FLASH2, 65, 0, 4),
     ("f3-T160-gemm", gen.FLASH3, 160, 2, 9),
     ("f3-T64-gemm", gen.FLASH3, 64, 2, 5),
+    ("c1-T20-gemv", gen.CODER1, 20, 1, 3),
+    ("c1-T200-gemm", gen.CODER1, 200, 2, 7),
 ]
 
 
@@ -383,3 +390,35 @@ def test_fused_decode_3bit_batch():
     sel = np.arange(0, T, 3, dtype=np.int32)
     _, ref, _, _ = oracle.moe_forward(layer_of(shape), xh, sel=sel, threads=THREADS)
     check_output(yf[sel], ref, "fused 3-bit T=64")
+
+
+@pytest.mark.parametrize("shape", [gen.FLASH2, gen.FLASH3, gen.CODER1], ids=["2bit", "3bit", "1bit"])
+def test_prefill_full_tiles(shape):
+    """T = 8192 at full tile sizes: the oracle checks the tokens of the hottest
+    expert's ragged last tile, the tokens on each side of every interior tile
+    boundary of that expert (positions 256 u - 2 .. 256 u + 1 in its token
+    list), every token of two mid-load experts, and the shared expert's tile
+    boundaries (tokens 256 u - 1, 256 u)."""
+    T, tile = 8192, 256
+    w = layer_of(shape)
+    x = gen.hidden(T, shape.hidden, seed=12)
+    L = gpu_layer(shape, T)
+    ridx, roff = check_route(L, w, x, T, "prefill full tiles")
+    y = from_dev_bf16(L.forward(to_dev_bf16(x)))
+    L.sync_status()
+    cnt = np.diff(roff)
+    hot = int(np.argmax(cnt))
+    assert cnt[hot] > tile, "the hottest expert must span several tiles"
+    hot_tokens = np.nonzero((ridx == hot).any(axis=1))[0]  # ascending = its list order
+    sel = set(hot_tokens[(len(hot_tokens) // tile) * tile:].tolist())  # ragged last tile
+    for u in range(1, (len(hot_tokens) + tile - 1) // tile):
+        sel |= set(hot_tokens[max(0, u * tile - 2):u * tile + 2].tolist())
+    order = np.argsort(cnt, kind="stable")
+    nz = order[cnt[order] > 0]
+    for e in (nz[len(nz) // 2], nz[len(nz) // 2 + 1]):   # two mid-load experts
+        sel |= set(np.nonzero((ridx == e).any(axis=1))[0].tolist())
+    for u in range(1, T // tile):
+        sel |= {u * tile - 1, u * tile}
+    sel = np.array(sorted(sel), dtype=np.int32)
+    _, ref, _, _ = oracle.moe_forward(w, x, sel=sel, threads=THREADS)
+    check_output(y[sel], ref, f"prefill full tiles ({len(sel)} tokens)")
