@@ -238,7 +238,8 @@ size_t carve_workspace(strata_moe *h, char *base) {
     h->xs = take(slots * H * 2);
     h->dsplit = (float *)take(T > (size_t)kSmallMaxT ? T * (size_t)h->router_rows * 4 : 0);
     h->fused_tok = max_units(64, (int)k, (int)E, 8);
-    h->fused_stride = h->fused_tok + 64 * (int)(H / 128);
+    // + 1: the launch's item claim counter (last entry of each set)
+    h->fused_stride = h->fused_tok + 64 * (int)(H / 128) + 1;
     h->fused_bar = (unsigned long long *)take(8);
     h->fused_cnt = (int *)take((size_t)2 * h->fused_stride * 4);
     h->xex = (int *)take(T * 4);

@@ -158,7 +158,10 @@ constexpr int kMiscAbort = 0, kMiscScan = 1 /* 33 */, kMiscNUnits = 34, kMiscUto
               kMiscGCnt = 40 /* kFMaxRing: warps done with the item in a slot */,
               kMiscMeta = 48 /* kFMaxRing */, kMiscPubN = 56, kMiscPubSeen = 57,
               kMiscWarpsDone = 58, kMiscCombN = 59, kMiscCombSeen = 60,
-              kMiscPubQ = 64 /* kPubQ */, kMiscCombQ = 128 /* kPubQ */;
+              kMiscPubQ = 64 /* kPubQ */, kMiscCombQ = 128 /* kPubQ */,
+              kMiscDownN = 192, kMiscDownEnd = 193, kMiscDownSeen = 194,
+              kMiscDownQ = 196 /* kDownQ */;
+constexpr int kDownQ = 32;  // claimed down items handed from the copy warp to the fetch warp
 
 // Named barrier 1: the compute warps.
 STRATA_DEV void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFCompute) : "memory"); }
@@ -402,14 +405,49 @@ STRATA_DEV __half token_operand(float x, int ex, int i) {
     const float v = x * pow2f(-ex);
     return __float2half_rn(kBits <= 2 ? v * magic_col_scale(i & 31) : v);
 }
+// The correction of one block: the four column groups (one factor each) are
+// summed in order, then combined: corr = sum over g of -c_g (sum of B in g).
 template <int kBits>
 STRATA_DEV float block_correction(const __nv_bfloat16 *blk, int ex) {
     float v = 0.0f;
-#pragma unroll 8
-    for (int kk = 0; kk < 32; kk++)
-        v = fmaf(-magic_col_corr(kk, kBits),
-                 __half2float(token_operand<kBits>(__bfloat162float(blk[kk]), ex, kk)), v);
+#pragma unroll
+    for (int gq = 0; gq < 4; gq++) {
+        float gs = 0.0f;
+#pragma unroll
+        for (int kk = 8 * gq; kk < 8 * gq + 8; kk++)
+            gs += __half2float(token_operand<kBits>(__bfloat162float(blk[kk]), ex, kk));
+        v = fmaf(-magic_col_corr(8 * gq, kBits), gs, v);
+    }
     return v;
+}
+
+// One staged block (32 columns) of a token by one thread: the expert operand
+// B = fp16(x 2^-ex s(k)) written to dst, and (magic form) the block's
+// correction, in the same order as block_correction.
+template <int kBits>
+STRATA_DEV void stage_block(const __nv_bfloat16 *src, __half *dst, int ex, float *corr) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    const float sc = pow2f(-ex);
+    float v = 0.0f;
+#pragma unroll
+    for (int gq = 0; gq < 4; gq++) {
+        const uint4 in = s4[gq];
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        const float f = kBits <= 2 ? magic_col_scale(8 * gq) : 1.0f;
+        uint32_t o[4];
+        float gs = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const __half2 h = __floats2half2_rn(bf16_lo(w[j]) * sc * f, bf16_hi(w[j]) * sc * f);
+            o[j] = *reinterpret_cast<const uint32_t *>(&h);
+            gs += __low2float(h);
+            gs += __high2float(h);
+        }
+        d4[gq] = make_uint4(o[0], o[1], o[2], o[3]);
+        v = fmaf(-magic_col_corr(8 * gq, kBits), gs, v);
+    }
+    if (kBits <= 2) *corr = v;
 }
 
 
@@ -756,9 +794,21 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
             item_counts(Ng, N2, ug0);
             const int W = Ng + N2;
             int kd = 0;
-            for (int it = cta; it < W && ok; it += G, pos++) {
+            // items are claimed from one counter per launch, in ascending
+            // order: gate/up slabs first, then down blocks, so within a CTA
+            // every gate/up item precedes every down item (every down wait
+            // ends) and a CTA that finishes early takes more work; the next
+            // claim is requested while this item's copies go out
+            unsigned long long b0;
+            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
+            int *claim = p.cnt + (size_t)((b0 / (2ull * (unsigned long long)G)) & 1ull) * p.cnt_stride +
+                         p.cnt_stride - 1;
+            int nxt = atomicAdd(claim, 1);
+            for (; nxt < W && ok; pos++) {
+                const int it = nxt;
                 ok = acquire(pos);
                 if (!ok) break;
+                nxt = atomicAdd(claim, 1);
                 const int slot = pos % p.ring;
                 if (it < Ng) {
                     const int u = ug0 + it / nsl;
@@ -766,7 +816,22 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                     issue_gu(slot, units[u].x, it % nsl);
                 } else {
                     const int d = it - Ng, u = d / ndn, e = units[u].x;
-                    vmisc[kMiscMeta + slot] = (kKindDown << 28) | (kd << 20) | d;
+                    // (kd mod 2 na keeps the buffer and its phase parity in 8 bits)
+                    vmisc[kMiscMeta + slot] = (kKindDown << 28) | ((kd % (2 * p.na)) << 20) | d;
+                    // hand the down block to the fetch warp (its activation rows)
+                    long long t0 = clock64();
+                    while (kd - vmisc[kMiscDownSeen] >= kDownQ) {
+                        if (*abort_flag || clock64() - t0 > p.budget) {
+                            atomicCAS(p.err, 0, kErrTimeout);
+                            *abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                    vmisc[kMiscDownQ + kd % kDownQ] = d;
+                    __threadfence_block();
+                    vmisc[kMiscDownN] = kd + 1;
                     kd++;
                     const uint8_t *wd = (e == E ? p.shared : p.routed + (size_t)e * p.expert_bytes) +
                                         2 * p.mat_bytes + (size_t)(d % ndn) * dn_bytes;
@@ -775,6 +840,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                                   &full[slot], pol);
                 }
             }
+            __threadfence_block();
+            vmisc[kMiscDownEnd] = 1;  // no more down blocks for the fetch warp
             // one end marker per group (completes its slot without bytes)
             for (int gq = 0; gq < kGroups && ok; gq++) {
                 ok = acquire(pos);
@@ -840,14 +907,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
     // Grid barrier(s), then the activation rows of this CTA's down blocks.
     if (warp == kWFetch) {
         grid_dependency_wait();
-        {
-            // run the top-k code once on stale logits while the router works, so
-            // its instructions are in this SM's caches when the routing needs them
-            int pe;
-            float pw;
-            warp_topk(p.logits, E, k, lane, pe, pw);
-            if (pe == 0x7fffffff && pw == 1.0f) misc[kMiscTmp] = 1;  // keeps the call
-        }
         if (lane != 0) return;
         unsigned long long b0;
         asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(b0) : "l"(p.bar) : "memory");
@@ -873,13 +932,28 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         if (ok) ok = fwait(dsp, 0, p, abort_flag);
         int issued = 0;
         if (ok) {
-            int Ng, N2, ug0;
-            item_counts(Ng, N2, ug0);
-            const int W = Ng + N2;
-            int first = cta;
-            if (first < Ng) first += ((Ng - first + G - 1) / G) * G;  // first down position
-            for (int it = first; it < W && ok; it += G, issued++) {
-                const int d = it - Ng, u = d / ndn, kd = issued, b = kd % p.na;
+            // this CTA's down blocks in the order the copy warp claimed them
+            for (;; issued++) {
+                int d = -1;
+                long long t0 = clock64();
+                while (true) {
+                    if (issued < vmisc[kMiscDownN]) {
+                        d = vmisc[kMiscDownQ + issued % kDownQ];
+                        break;
+                    }
+                    if (vmisc[kMiscDownEnd] && issued >= vmisc[kMiscDownN]) break;
+                    if (*abort_flag || clock64() - t0 > p.budget) {
+                        atomicCAS(p.err, 0, kErrTimeout);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+                if (d < 0) break;
+                __threadfence_block();
+                vmisc[kMiscDownSeen] = issued + 1;  // the entry may be reused
+                const int u = d / ndn, kd = issued, b = kd % p.na;
                 const int4 un = units[u];
                 // buffer b is free once the group's warps are done with its last block
                 if (kd >= p.na && !(ok = fwait(&aempty[b], ((kd / p.na) - 1) & 1, p, abort_flag)))
@@ -1188,19 +1262,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
             }
         } else if (alive && staged) {
             const int t0 = tid - 32 * T, nt = kFCompute - 32 * T;
-            for (int i = t0; i < T * (H / 2); i += nt) {
-                const int t = i / (H / 2), c = 2 * (i % (H / 2));
-                const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(xb + (size_t)t * H + c);
-                __half2 h;
-                h.x = token_operand<kBits>(__bfloat162float(v.x), sex[t], c);
-                h.y = token_operand<kBits>(__bfloat162float(v.y), sex[t], c + 1);
-                *reinterpret_cast<__half2 *>(xs + (size_t)t * (H + 8) + c) = h;
+            for (int task = t0; task < T * nbh; task += nt) {
+                const int t = task / nbh, b = task % nbh;
+                stage_block<kBits>(xb + (size_t)t * H + 32 * b, xs + (size_t)t * (H + 8) + 32 * b,
+                                   sex[t], scorr + t * nbh + b);
             }
-            if (kMagic)
-                for (int task = t0; task < T * nbh; task += nt) {
-                    const int t = task / nbh, b = task % nbh;
-                    scorr[t * nbh + b] = block_correction<kBits>(xb + (size_t)t * H + 32 * b, sex[t]);
-                }
         }
         if (!alive && lane == 0) misc[kMiscDead] = 1;
         compute_sync();

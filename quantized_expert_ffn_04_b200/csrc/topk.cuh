@@ -51,24 +51,41 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[16], uint32_t &b
     bq = l ? q2[0] : q2[1];
 }
 
-// Top-k of one token by one warp (E <= 512: lane l holds logits l, l+32, ...).
-// Each round takes the largest key over the warp (redux.sync max) and, among
-// the lanes holding it, the lowest expert id (redux.sync min), i.e. the larger
-// logit and on equal logits the lower id; the winning lane drops that entry
-// and finds its next best.  Lane j < k ends with pick j and its weight
+// Top-k of one token by one warp (E <= 512: lane l holds the logits of
+// experts 16 l .. 16 l + 15, read with four 16-byte loads when E is a multiple
+// of 4).  Each round takes the largest key over the warp (redux.sync max) and,
+// among the lanes holding it, the lowest expert id (redux.sync min), i.e. the
+// larger logit and on equal logits the lower id; the winning lane drops that
+// entry and finds its next best.  Lane j < k ends with pick j and its weight
 // exp(l_j - m) / sum.
 static __device__ __noinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
-                                        int &pick_e, float &pick_w) {
+                                              int &pick_e, float &pick_w) {
     uint32_t key[16];
-    // every load is unconditional (entries past E re-read the last one) and
-    // its value is used unconditionally (masked, not branched on), so the
-    // compiler cannot sink the loads into branches: the 16 are in flight
-    // together instead of one after another
+    const int e0 = 16 * lane;
+    // every load is unconditional (entries past E re-read valid ones) and its
+    // value is used unconditionally (masked), so no load waits for another
+    if ((E & 3) == 0) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(row);
+        float4 v[4];
 #pragma unroll
-    for (int q = 0; q < 16; q++) {
-        const int e = q * 32 + lane;
-        const float v = __ldcg(row + (e < E ? e : E - 1));
-        key[q] = logit_key(v) & (0u - (uint32_t)(e < E));
+        for (int i = 0; i < 4; i++) {
+            const int e = e0 + 4 * i;
+            v[i] = __ldcg(r4 + ((e < E ? e : E - 4) >> 2));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float f[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                key[4 * i + j] = logit_key(f[j]) & (0u - (uint32_t)(e0 + 4 * i + j < E));
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 16; q++) {
+            const int e = e0 + q;
+            const float v = __ldcg(row + (e < E ? e : E - 1));
+            key[q] = logit_key(v) & (0u - (uint32_t)(e < E));
+        }
     }
     uint32_t bk;
     int bq;
@@ -77,14 +94,14 @@ static __device__ __noinline__ void warp_topk(const float *__restrict__ row, int
     int my_e = -1;
     for (int j = 0; j < k; j++) {
         const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t cand = (bk == wk && bk != 0u) ? (uint32_t)(bq * 32 + lane) : 0xffffffffu;
+        const uint32_t cand = (bk == wk && bk != 0u) ? (uint32_t)(e0 + bq) : 0xffffffffu;
         const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
         if (lane == j) {
             my_k = wk;
             my_e = (int)we;
         }
-        if ((int)(we & 31u) == lane) {
-            const int wq = (int)(we >> 5);
+        if ((int)(we >> 4) == lane) {
+            const int wq = (int)(we & 15u);
 #pragma unroll
             for (int q = 0; q < 16; q++) key[q] = q == wq ? 0u : key[q];
             lane_best(key, bk, bq);
