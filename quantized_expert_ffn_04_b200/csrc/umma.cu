@@ -414,9 +414,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                 if (kGateUp) {
                     float uv[32];
                     tmem_ld32(tb + kTN + nc * 32, uv);
-                    // lane j holds the prescale exponent of column j of the chunk
+                    // lane j holds the prescale exponent of column j of the chunk;
+                    // when the chunk's columns share one (the usual case) the
+                    // factor is taken once, without a shuffle per element
                     const int exl = lane < cnt ? __ldg(p.slot_ex + slot0 + nc * 32 + lane) : 0;
-                    if (cnt >= 32) {
+                    const int ex0 = __shfl_sync(0xffffffffu, exl, 0);
+                    if (__all_sync(0xffffffffu, lane >= cnt || exl == ex0)) {
+                        const float f = pow2f(ex0);
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (j < cnt)
+                                p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(
+                                    __fdividef(gv[j], 1.0f + __expf(-(gv[j] * f))) * uv[j]);
+                    } else if (cnt >= 32) {
 #pragma unroll
                         for (int j = 0; j < 32; j++)
                             p.out[o0 + (size_t)j * p.out_ld] = __float2half_rn(
