@@ -1011,7 +1011,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                     late = 1;
                 }
                 if (__shfl_sync(0xffffffffu, late, 0)) break;
-                __nanosleep(500);
+                __nanosleep(100);
                 continue;
             }
             __syncwarp();
