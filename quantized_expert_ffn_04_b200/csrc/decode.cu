@@ -67,7 +67,9 @@ namespace strata {
 
 constexpr int kFWarps = 16;                     // compute warps
 constexpr bool kFExtras = false;                // shared-expert slabs before routing
-constexpr int kGroups = 2, kGWarps = 8;         // two groups of 8 take alternate ring positions
+constexpr int kGWarps = 4;                      // warps of a compute group (one item at a time)
+constexpr int kGroups = kFWarps / kGWarps;      // the groups take ring positions in turn
+constexpr int kDH = kGWarps / 4;                // K splits of a down block's slab pairs
 constexpr int kFCompute = 32 * kFWarps;         // compute threads
 constexpr int kWCopy = kFWarps, kWPub = kFWarps + 1, kWFetch = kFWarps + 2, kWComb = kFWarps + 3;
 constexpr int kFThreads = 32 * (kFWarps + 4);
@@ -546,7 +548,7 @@ auto last_warp = [&](int slot) -> bool {
         if (kind != kKindDown) {
             // ---------------------------------- gate/up slab, K eighth q
             // pairs of blocks: every range starts at an even block
-            const int b0 = 2 * (q * (nbh / 2) / 8), b1 = 2 * ((q + 1) * (nbh / 2) / 8);
+            const int b0 = 2 * (q * (nbh / 2) / kGWarps), b1 = 2 * ((q + 1) * (nbh / 2) / kGWarps);
             // the lane's two token columns (columns past n repeat token 0)
             const int ta = slot_tok(slot0 + (2 * cq < n ? 2 * cq : 0));
             const int tb = slot_tok(slot0 + (2 * cq + 1 < n ? 2 * cq + 1 : 0));
@@ -609,15 +611,15 @@ auto last_warp = [&](int slot) -> bool {
                 vmisc[kMiscPubQ + idx % kPubQ] = u + 1;
             }
         } else {
-            // ------------------ down block: slabs 2 (q >> 1) + {0, 1}, K half q & 1
+            // ---- down block: slabs 2 (q / kDH) + {0, 1}, K part q % kDH of kDH
             const int kd = (meta >> 20) & 0xff, b = kd % p.na;
             if (!warp_fwait(&abar[b], (kd / p.na) & 1, p, abort_flag, lane)) return -1;
             const __half *abuf = abuf0 + (size_t)b * kFTile * (p.Ip + 8);
-            const int ar = lane & 7, pr = q >> 1, h = q & 1;
+            const int ar = lane & 7, pr = q / kDH, h = q % kDH;
             const __half *rowp = abuf + (size_t)(ar < n ? ar : 0) * (p.Ip + 8);
             const uint8_t *s0 = w + (size_t)(2 * pr) * p.nseg_i * UB;
             slab2_blocks<kBits, kSrcSmem, false>(a0, a1, s0, s0 + (size_t)p.nseg_i * UB,
-                                                 2 * (h * (nbi / 2) / 2), 2 * ((h + 1) * (nbi / 2) / 2), rowp, nullptr,
+                                                 2 * (h * (nbi / 2) / kDH), 2 * ((h + 1) * (nbi / 2) / kDH), rowp, nullptr,
                                                  nullptr, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&aempty[b]);  // activation rows consumed
@@ -629,16 +631,21 @@ auto last_warp = [&](int slot) -> bool {
                 if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
                 continue;
             }
-            // the last warp: both K halves of every slab, in a fixed order
+            // the last warp: the K parts of every slab, in a fixed order
 #pragma unroll
             for (int pp = 0; pp < kDownSlabs / 2; pp++) {
-                const float4 *r0 = reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp) * 32 + lane) * 8);
-                const float4 *r1 =
-                    reinterpret_cast<const float4 *>(rd + ((size_t)(2 * pp + 1) * 32 + lane) * 8);
 #pragma unroll
                 for (int sl = 0; sl < 2; sl++) {
-                    const float4 v0 = r0[sl], v1 = r1[sl];
-                    const float yv[4] = {v0.x + v1.x, v0.y + v1.y, v0.z + v1.z, v0.w + v1.w};
+                    float yv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int hh = 0; hh < kDH; hh++) {
+                        const float4 v = reinterpret_cast<const float4 *>(
+                            rd + ((size_t)(kDH * pp + hh) * 32 + lane) * 8)[sl];
+                        yv[0] += v.x;
+                        yv[1] += v.y;
+                        yv[2] += v.z;
+                        yv[3] += v.w;
+                    }
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
                         const int tok = 2 * cq + (i & 1);
@@ -1426,7 +1433,7 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     // partial-sum area also holds the router's copy of staged token rows
     const int slot_bytes = p.item_bytes + kRedSlot;
     const int xi_slots = (align16(T * g.H * 2) + kRedSlot - 1) / kRedSlot;
-    p.na = 2;
+    p.na = kGroups < kMaxA ? kGroups : kMaxA;  // one activation buffer per group
     p.staged = (T <= kFStagedMaxT && g_fused_max_smem - total(0, 1, p.na) >=
                                          (xi_slots > 4 ? xi_slots : 4) * slot_bytes)
                    ? 1 : 0;
