@@ -33,19 +33,18 @@
 //     deterministic), for T > 16 tokens the top-k is split over CTAs with a
 //     second barrier;
 //   * items: the list [routed gate/up slabs (unit, 16 rows)] + [down blocks
-//     (unit, 128 rows)] is dealt out round-robin over the CTAs, so at every
-//     step all CTAs work on neighbouring units: a unit's gate/up slabs are
-//     all done long before its down blocks come up, and no item is claimed
-//     with an atomic;
-//   * two groups of 8 compute warps take alternate ring positions; the 8
-//     warps of a group each take a share of the item (an eighth of K of both
-//     the gate and the up slab; two slabs and half of K of a down block, so
-//     one token fragment serves two slabs) and run independently: no barrier
-//     inside the item loop, and a ring slot is free as soon as its last warp
-//     is done, so most of the ring is in flight; the last warp to finish an
-//     item completes it (sums the partial products in a fixed order and
-//     applies SwiGLU, or stores the block's rows and counts them for the
-//     combine);
+//     (unit, 128 rows)] is claimed item by item from one counter per launch
+//     (two counter sets alternate by launch parity), so all CTAs work on
+//     neighbouring units, a unit's gate/up slabs are all done long before
+//     its down blocks come up, and a CTA that finishes early takes more;
+//   * four groups of 4 compute warps take ring positions in turn; the 4
+//     warps of a group each take a share of the item (a quarter of K of both
+//     the gate and the up slab; two slabs of a down block, so one token
+//     fragment serves both) and run independently: no barrier inside the
+//     item loop, and a ring slot is free as soon as its last warp is done,
+//     so most of the ring is in flight; the last warp to finish an item
+//     completes it (sums the partial products in a fixed order and applies
+//     SwiGLU, or stores the block's rows and counts them for the combine);
 //   * the publish warp turns finished gate/up slabs into per-unit counts
 //     (one gpu-scope fence per batch), and the fetch warp waits for the
 //     counts a down block needs and copies that unit's activation rows in,
@@ -453,15 +452,15 @@ STRATA_DEV void stage_block(const __nv_bfloat16 *src, __half *dst, int ex, float
 }
 
 
-// The ring items of one compute warp: its group's positions jpos, jpos + 2,
-// ... up to `stop`.  Returns the next position, or -1 once the end marker is
+// The ring items of one compute warp: its group's positions jpos,
+// jpos + kGroups, ... up to `stop`.  Returns the next position, or -1 once the end marker is
 // seen or the launch aborts.  One non-inlined copy serves both calls (the
 // shared expert's slabs before routing, then the routed items), so the hot
 // loop exists once per kernel instantiation and stays in the instruction
 // caches next to the other roles' loops.
-//   gate/up slab: warp q of the group takes an eighth of K of both the gate
-//   and the up slab; down block: warp q the slabs 2 (q >> 1), 2 (q >> 1) + 1,
-//   half of K; the last of the group's 8 warps to finish an item completes it.
+//   gate/up slab: warp q of the group takes a quarter of K of both the gate
+//   and the up slab; down block: warp q the slabs 2q and 2q + 1, all of K; the
+//   last of the group's 4 warps to finish an item completes it.
 template <int kBits, bool kStaged>
 __device__ __noinline__ int fused_run_items(const FusedParams &p, int jpos, int stop) {
     extern __shared__ __align__(128) uint8_t sm[];
@@ -546,7 +545,7 @@ auto last_warp = [&](int slot) -> bool {
         float *rd = red + (size_t)slot * (kRedSlot / 4);  // [warp of group][lane][8]
         float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
         if (kind != kKindDown) {
-            // ---------------------------------- gate/up slab, K eighth q
+            // ---------------------------------- gate/up slab, K quarter q
             // pairs of blocks: every range starts at an even block
             const int b0 = 2 * (q * (nbh / 2) / kGWarps), b1 = 2 * ((q + 1) * (nbh / 2) / kGWarps);
             // the lane's two token columns (columns past n repeat token 0)
@@ -571,7 +570,7 @@ auto last_warp = [&](int slot) -> bool {
                 if (lane == 0) mbar_arrive(&empty[slot]);  // weights consumed
                 continue;
             }
-            // the last warp: the K eighths in a fixed order, then SwiGLU
+            // the last warp: the K quarters in a fixed order, then SwiGLU
             float gs[4] = {0.f, 0.f, 0.f, 0.f}, us[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < kGWarps; j++) {
