@@ -1368,11 +1368,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
 static int g_fused_max_smem = 0;
 static int g_fused_sms = 0;
 
-int fused_decode_supported(const Geometry &g, int T) {
-    return T >= 1 && T <= kFMaxT && g.E <= 512 && g.k <= kFMaxK && g.H % 128 == 0 &&
-           g.Ip % 128 == 0 && g.H <= 8192;
-}
-
 size_t fused_item_bytes(const Geometry &g) {
     const int a = 2 * g.nseg_h, b = kDownSlabs * g.nseg_i;
     return (size_t)(a > b ? a : b) * g.ub;
@@ -1380,9 +1375,55 @@ size_t fused_item_bytes(const Geometry &g) {
 
 int fused_grid() { return g_fused_sms; }
 
+// Shared-memory plan of a launch: whether the token rows are staged, the
+// activation buffers and the ring depth.  The groups take ring positions in
+// turn and wait on a slot's barrier by phase parity, so the wait for position
+// p is unambiguous only if position p - ring (the slot's previous fill) was
+// waited for already, by this group: ring >= kGroups.  Likewise one activation
+// buffer per group.  Returns false when the shape does not fit.
+struct FusedPlan {
+    int staged, na, ring, units_max, item_bytes;
+};
+static bool fused_plan(const Geometry &g, int T, FusedPlan &pl) {
+    if (!(T >= 1 && T <= kFMaxT && g.E <= 512 && g.k <= kFMaxK && g.H % 128 == 0 &&
+          g.Ip % 128 == 0 && g.H <= 8192) ||
+        g_fused_max_smem == 0 || g_fused_sms == 0)
+        return false;
+    pl.item_bytes = (int)fused_item_bytes(g);
+    pl.units_max = max_units(T, g.k, g.E, kFTile);
+    auto total = [&](int ring, int staged, int na) {
+        return fused_smem(T, g.E, g.k, g.H, g.Ip, ring, pl.item_bytes, staged, pl.units_max, na)
+            .total;
+    };
+    // the router slice of the CTA with the most experts must fit the ring
+    const int G = g_fused_sms;
+    const int ne_max = (g.E + G - 1) / G;
+    const int nwc = (ne_max * g.H * 4 + pl.item_bytes - 1) / pl.item_bytes;
+    // a ring slot costs its item bytes plus the partial sums of the warps; the
+    // partial-sum area also holds the router's copy of staged token rows
+    const int slot_bytes = pl.item_bytes + kRedSlot;
+    const int xi_slots = (align16(T * g.H * 2) + kRedSlot - 1) / kRedSlot;
+    pl.na = kGroups;
+    if (pl.na > kMaxA) return false;
+    const int min_ring = kGroups > nwc + 1 ? kGroups : nwc + 1;
+    // staging the token rows needs room for its router copy and a full ring
+    const int need_staged = (xi_slots > kGroups ? xi_slots : kGroups) * slot_bytes;
+    pl.staged = (T <= kFStagedMaxT && g_fused_max_smem - total(0, 1, pl.na) >= need_staged) ? 1 : 0;
+    pl.ring = (g_fused_max_smem - total(0, pl.staged, pl.na)) / slot_bytes;
+    if (pl.ring > kFMaxRing) pl.ring = kFMaxRing;
+    if (pl.staged && pl.ring < xi_slots) return false;
+    return pl.ring >= min_ring;
+}
+
+int fused_decode_supported(const Geometry &g, int T) {
+    FusedPlan pl;
+    return fused_plan(g, T, pl) ? 1 : 0;
+}
+
 cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const FusedArgs &fa,
                                 int T, cudaStream_t s) {
-    if (!fused_decode_supported(g, T) || g_fused_max_smem == 0) return cudaErrorInvalidValue;
+    FusedPlan pl;
+    if (!fused_plan(g, T, pl)) return cudaErrorInvalidValue;
     FusedParams p{};
     p.x = reinterpret_cast<const __nv_bfloat16 *>(fa.x);
     p.Wp = reinterpret_cast<const float4 *>(fa.router_wp);
@@ -1398,8 +1439,8 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     p.Ip = g.Ip;
     p.nseg_h = g.nseg_h;
     p.nseg_i = g.nseg_i;
-    p.item_bytes = (int)fused_item_bytes(g);
-    p.units_max = max_units(T, g.k, g.E, kFTile);
+    p.item_bytes = pl.item_bytes;
+    p.units_max = pl.units_max;
     p.cnt_tok = fa.cnt_tok;
     p.w2 = fa.w2;
     p.logits = fa.logits;
@@ -1418,32 +1459,11 @@ cudaError_t launch_fused_decode(const Geometry &g, const ExpertWeights &w, const
     p.err = fa.err;
     p.budget = fa.budget;
     const int G = g_fused_sms;
-    // the router slice of the CTA with the most experts must fit the ring
-    const int ne_max = (g.E + G - 1) / G;
-    const int wb = ne_max * g.H * 4;
-    // shared memory: staging of the token rows, then activation buffers and
-    // as deep a ring as fits
-    const int xs_bytes = align16(T * (g.H + 8) * 2);
-    auto total = [&](int ring, int staged, int na) {
-        return fused_smem(T, g.E, g.k, g.H, g.Ip, ring, p.item_bytes, staged, p.units_max, na)
-            .total;
-    };
-    // a ring slot costs its item bytes plus the partial sums of the warps; the
-    // partial-sum area also holds the router's copy of staged token rows
-    const int slot_bytes = p.item_bytes + kRedSlot;
-    const int xi_slots = (align16(T * g.H * 2) + kRedSlot - 1) / kRedSlot;
-    p.na = kGroups < kMaxA ? kGroups : kMaxA;  // one activation buffer per group
-    p.staged = (T <= kFStagedMaxT && g_fused_max_smem - total(0, 1, p.na) >=
-                                         (xi_slots > 4 ? xi_slots : 4) * slot_bytes)
-                   ? 1 : 0;
-    (void)xs_bytes;
-    const int room = g_fused_max_smem - total(0, p.staged, p.na);
-    p.ring = room / slot_bytes;
-    if (p.ring > kFMaxRing) p.ring = kFMaxRing;
-    if (p.staged && p.ring < xi_slots) return cudaErrorInvalidValue;
-    const int nwc = (wb + p.item_bytes - 1) / p.item_bytes;
-    if (p.ring < 2 || nwc >= p.ring) return cudaErrorInvalidValue;
-    const int smem = total(p.ring, p.staged, p.na);
+    p.staged = pl.staged;
+    p.na = pl.na;
+    p.ring = pl.ring;
+    const int smem = fused_smem(T, g.E, g.k, g.H, g.Ip, p.ring, p.item_bytes, p.staged, p.units_max,
+                                p.na).total;
     auto kern = g.bits == 1   ? (p.staged ? fused_decode_kernel<1, true> : fused_decode_kernel<1, false>)
                 : g.bits == 2 ? (p.staged ? fused_decode_kernel<2, true> : fused_decode_kernel<2, false>)
                               : (p.staged ? fused_decode_kernel<3, true> : fused_decode_kernel<3, false>);
