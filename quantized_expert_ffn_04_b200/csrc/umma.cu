@@ -399,11 +399,19 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         int it = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, it++) {
             const int buf = it % NB, use = it / NB;
-            if (!pipe_wait(&acc_full[buf], use & 1, p.budget, p.err, abort_flag)) break;
-            tc_fence_after();
+            // the tile's unit and (gate/up) the prescale exponents of its
+            // columns are requested before the wait for the accumulators, so
+            // their latency hides behind the tile's MMAs: lane j holds the
+            // exponent of column 32 c + j in exr[c]
             const int rt = t % p.n_rt;
             const int4 un = tile_unit(p, t / p.n_rt);
             const int slot0 = un.y, n = un.z;
+            int exr[kTN / 32];
+#pragma unroll
+            for (int c = 0; c < kTN / 32; c++)
+                exr[c] = kGateUp && 32 * c + lane < n ? __ldg(p.slot_ex + slot0 + 32 * c + lane) : 0;
+            if (!pipe_wait(&acc_full[buf], use & 1, p.budget, p.err, abort_flag)) break;
+            tc_fence_after();
             const int row = rt * kTM + r_in;
             const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + buf * kTN;
             for (int nc = 0; nc * 32 < n; nc++) {
@@ -417,7 +425,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
                     // lane j holds the prescale exponent of column j of the chunk;
                     // when the chunk's columns share one (the usual case) the
                     // factor is taken once, without a shuffle per element
-                    const int exl = lane < cnt ? __ldg(p.slot_ex + slot0 + nc * 32 + lane) : 0;
+                    int exl = 0;
+#pragma unroll
+                    for (int c = 0; c < kTN / 32; c++) exl = c == nc ? exr[c] : exl;
                     const int ex0 = __shfl_sync(0xffffffffu, exl, 0);
                     if (__all_sync(0xffffffffu, lane >= cnt || exl == ex0)) {
                         const float f = pow2f(ex0);
