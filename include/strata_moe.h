@@ -265,7 +265,10 @@ enum {
                                    kernel where it applies, else the decode GEMV chain; larger T
                                    the prefill GEMM), 1 force the decode GEMV kernel chain,
                                    2 force the prefill GEMM, 3 force the fused decode kernel
-                                   (T <= 64, E <= 512; forward fails otherwise) */
+                                   (T <= 64, E <= 512, k <= 16, H and I multiples of 128, and
+                                   its shared-memory plan must give every compute group a ring
+                                   slot; auto mode takes the chain for shapes that do not fit,
+                                   a forced forward fails with STRATA_ERR_INVALID_ARG) */
     STRATA_OPT_WAIT_BUDGET = 2, /* bound of every device-side wait, in SM clock cycles
                                    (default 4e9); 0 makes every wait give up at once */
     STRATA_OPT_DECODE_MAX_T = 3 /* largest T run by the decode kernels in auto mode (default 64) */
