@@ -507,8 +507,8 @@ def run_own(args, wl, emit=True, extra=None):
     return line
 
 
-# Workloads measured briefly alongside the default one (one GPU only), so
-# the default line also carries the other decode shapes and the prefill:
+# Workloads measured briefly after the default one (one GPU only), so the
+# default line also carries the other decode shapes and the prefill:
 # (workload, timed steps, layers rotated)
 ALSO = [("decode-t1", 400, 8), ("decode3-t64", 100, 8), ("pruned256-t4", 400, 8),
         ("coder1-t4", 400, 8), ("prefill-t8192", 20, 4), ("coder1-t8192", 20, 4)]
@@ -720,12 +720,14 @@ def main():
         run_reference(args, args.workload)
     elif args.workload.startswith("stack"):
         run_stack(args, args.workload)
+    elif (args.workload == DEFAULT_WORKLOAD and not args.no_also and args.gpus == 1
+            and int(os.environ.get("WORLD_SIZE", "1")) == 1):
+        # the headline first; the short runs after it can only add to its line
+        line = run_own(args, args.workload, emit=False)
+        line["other_workloads"] = run_also(args)
+        print(json.dumps(line), flush=True)
     else:
-        extra = None
-        if (args.workload == DEFAULT_WORKLOAD and not args.no_also and args.gpus == 1
-                and int(os.environ.get("WORLD_SIZE", "1")) == 1):
-            extra = {"other_workloads": run_also(args)}
-        run_own(args, args.workload, extra=extra)
+        run_own(args, args.workload)
 
 
 if __name__ == "__main__":

@@ -68,3 +68,37 @@ def test_traffic_records_apply_only_to_their_sources():
         got = bench.traffic_from_profile(wl)
         assert got == (d["dram_bytes_per_launch"] if same else None)
     assert found >= 1
+
+
+def test_default_line_prints_once_with_the_short_runs(monkeypatch, capsys):
+    calls = []
+
+    def fake_run_own(a, wl, emit=True, extra=None):
+        calls.append((wl, emit))
+        if wl == "prefill-t8192":
+            raise RuntimeError("out of memory")
+        line = {"metric": "MoE-layer tokens/s", "value": 3.0, "ms_per_step": 1.0,
+                "clocks": {"sm_mhz": 1965.0},
+                "roofline": {"launch_ms": 0.5, "frac": 0.25, "unit": "GB/s", "peak": 6650.0}}
+        if emit:
+            print(json.dumps(line))
+        return line
+
+    monkeypatch.setattr(bench, "run_own", fake_run_own)
+    monkeypatch.setattr("sys.argv", ["bench.py"])
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.main()
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["value"] == 3.0
+    assert calls[0] == (bench.DEFAULT_WORKLOAD, False)  # the headline runs first
+    assert "out of memory" in d["other_workloads"]["prefill-t8192"]["error"]
+    assert d["other_workloads"]["decode-t1"]["value"] == 3.0
+    # --no-also: the headline alone
+    calls.clear()
+    monkeypatch.setattr("sys.argv", ["bench.py", "--no-also"])
+    bench.main()
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and "other_workloads" not in json.loads(lines[0])
+    assert calls == [(bench.DEFAULT_WORKLOAD, True)]
